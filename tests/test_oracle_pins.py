@@ -1,0 +1,352 @@
+"""Pins for the CPU oracle: values and properties fixed by the pages and by the
+mathematics, chosen so that a dropped term, a wrong sign or index, or a
+transposed operand in the oracle fails at least one of them."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import read_golden
+
+RNG = np.random.default_rng(12345)
+
+
+def _rand(*shape):
+    return RNG.standard_normal(shape)
+
+
+# ---------------------------------------------------------------------------
+# Worked examples printed on the pages
+# ---------------------------------------------------------------------------
+
+def test_two_tile_example_intermediates():
+    g = read_golden("two_tile_example.txt")
+    out, lse, hist = oracle.online_softmax_row(g["scores"], g["values"], int(g["tile"]))
+    m1, l1, u1, _ = hist[0]
+    nd = int(g["decimals"])
+    assert m1 == g["after_tile1_m"]
+    assert round(l1, nd) == g["after_tile1_l"]
+    assert round(u1, nd) == g["after_tile1_u"]
+    # The page's closed forms for the state after tile 2.
+    l2 = math.exp(-1) * (1 + math.exp(-1)) + 1 + math.exp(-3)
+    u2 = math.exp(-1) * (10 + 20 * math.exp(-1)) + 30 + 40 * math.exp(-3)
+    m_final, l_final, u_final, _ = hist[1]
+    assert m_final == 3.0
+    assert math.isclose(l_final, l2, rel_tol=1e-14)
+    assert math.isclose(u_final, u2, rel_tol=1e-14)
+    # The page's assertion: the tiled result equals the full-row softmax, rel 1e-12.
+    assert math.isclose(out, u2 / l2, rel_tol=1e-12)
+    assert math.isclose(lse, 3.0 + math.log(l2), rel_tol=1e-14)
+
+
+def test_two_tile_example_through_attention_definition():
+    """The same row as a 1-query attention with d=1, q=1, keys=scores, scale=1."""
+    g = read_golden("two_tile_example.txt")
+    l2 = math.exp(-1) * (1 + math.exp(-1)) + 1 + math.exp(-3)
+    u2 = math.exp(-1) * (10 + 20 * math.exp(-1)) + 30 + 40 * math.exp(-3)
+    q = np.ones((1, 1, 1, 1))
+    k = np.array(g["scores"]).reshape(1, 4, 1, 1)
+    v = np.array(g["values"]).reshape(1, 4, 1, 1)
+    O, LSE = oracle.attention_forward(q, k, v, 1.0, False)
+    assert math.isclose(O[0, 0, 0, 0], u2 / l2, rel_tol=1e-12)
+    assert math.isclose(O[0, 0, 0, 0], 24.71148648358232, rel_tol=1e-12)
+    assert math.isclose(LSE[0, 0, 0], 3.0 + math.log(l2), rel_tol=1e-14)
+
+
+def test_eight_key_example_every_tile_size():
+    g = read_golden("eight_key_example.txt")
+    nd = int(g["decimals"])
+    out4, _, hist = oracle.online_softmax_row(g["scores"], g["values"], int(g["tile"]))
+    assert hist[0][0] == g["after_tile1_max"]
+    assert round(hist[0][3], nd) == g["after_tile1_output"]
+    assert round(out4, nd) == g["final_output"]
+    outs = []
+    for tile in range(1, 9):
+        o, lse, _ = oracle.online_softmax_row(g["scores"], g["values"], tile)
+        assert round(o, nd) == g["final_output"]
+        outs.append((o, lse))
+    ref_o, ref_lse = oracle.brute_force_row(g["scores"], g["values"])
+    for o, lse in outs:
+        assert math.isclose(o, ref_o, rel_tol=1e-13)
+        assert math.isclose(lse, ref_lse, rel_tol=1e-13)
+    # and the attention definition agrees
+    q = np.ones((1, 1, 1, 1))
+    k = np.array(g["scores"]).reshape(1, 8, 1, 1)
+    v = np.array(g["values"]).reshape(1, 8, 1, 1)
+    O, LSE = oracle.attention_forward(q, k, v, 1.0, False)
+    assert round(O[0, 0, 0, 0], nd) == g["final_output"]
+    assert math.isclose(LSE[0, 0, 0], ref_lse, rel_tol=1e-14)
+
+
+def test_online_softmax_vector_values_match_definition():
+    s = _rand(37) * 3
+    vals = _rand(37, 5)
+    ref_w = np.exp(s - s.max())
+    ref = (ref_w[:, None] * vals).sum(0) / ref_w.sum()
+    for tile in (1, 3, 8, 37, 64):
+        o, lse, _ = oracle.online_softmax_row(s, vals, tile)
+        np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-13)
+        assert math.isclose(lse, s.max() + math.log(ref_w.sum()), rel_tol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Brute force on tiny inputs (pure-Python loops), including the causal rule
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("Tq,Tk,causal", [(5, 5, False), (5, 5, True), (3, 6, True), (1, 4, True)])
+def test_forward_matches_brute_force(Tq, Tk, causal):
+    d = 3
+    q, k, v = _rand(1, Tq, 1, d), _rand(1, Tk, 1, d), _rand(1, Tk, 1, d)
+    s = 0.7
+    O, LSE = oracle.attention_forward(q, k, v, s, causal)
+    for i in range(Tq):
+        keys = [j for j in range(Tk) if (not causal) or j <= i + Tk - Tq]
+        scores = [s * sum(q[0, i, 0, c] * k[0, j, 0, c] for c in range(d)) for j in keys]
+        for c in range(d):
+            o, lse = oracle.brute_force_row(scores, [v[0, j, 0, c] for j in keys])
+            assert math.isclose(O[0, i, 0, c], o, rel_tol=1e-12, abs_tol=1e-13)
+        assert math.isclose(LSE[0, 0, i], lse, rel_tol=1e-13)
+
+
+def test_causal_rule_position_three():
+    """A query at position 3 uses columns 0..3 and ignores 4 and later."""
+    assert [j for j in range(8) if oracle.causal_visible(3, j, 8, 8)] == [0, 1, 2, 3]
+    # changing a future key/value must not change row 3
+    q, k, v = _rand(1, 8, 1, 4), _rand(1, 8, 1, 4), _rand(1, 8, 1, 4)
+    O1, L1 = oracle.attention_forward(q, k, v, 0.5, True)
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 4:] += 10.0
+    v2[0, 4:] -= 3.0
+    O2, L2 = oracle.attention_forward(q, k2, v2, 0.5, True)
+    np.testing.assert_array_equal(O1[0, :4], O2[0, :4])
+    np.testing.assert_array_equal(L1[0, 0, :4], L2[0, 0, :4])
+    assert not np.allclose(O1[0, 4:], O2[0, 4:])
+
+
+# ---------------------------------------------------------------------------
+# Invariants and degenerate cases
+# ---------------------------------------------------------------------------
+
+def test_probability_rows_sum_to_one_and_dv_sum():
+    B, T, H, d = 2, 9, 2, 4
+    q, k, v, do = _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d)
+    for causal in (False, True):
+        # P rows sum to 1: O of V = all-ones is all-ones
+        O, _ = oracle.attention_forward(q, k, np.ones_like(v), 0.3, causal)
+        np.testing.assert_allclose(O, 1.0, rtol=0, atol=1e-14)
+        # sum_j dV_j = sum_i dO_i because P is row-stochastic
+        _, _, dv = oracle.attention_backward(q, k, v, do, 0.3, causal)
+        np.testing.assert_allclose(dv.sum(axis=1), do.sum(axis=1), rtol=1e-12, atol=1e-12)
+
+
+def test_equal_scores_give_mean_of_values():
+    T, d = 7, 3
+    q = np.zeros((1, T, 1, d))
+    k, v = _rand(1, T, 1, d), _rand(1, T, 1, d)
+    O, LSE = oracle.attention_forward(q, k, v, 0.9, False)
+    np.testing.assert_allclose(O[0, :, 0], np.broadcast_to(v[0, :, 0].mean(0), (T, d)), rtol=1e-13)
+    np.testing.assert_allclose(LSE[0, 0], math.log(T), rtol=1e-14)
+    O, LSE = oracle.attention_forward(q, k, v, 0.9, True)
+    for i in range(T):
+        np.testing.assert_allclose(O[0, i, 0], v[0, :i + 1, 0].mean(0), rtol=1e-12, atol=1e-14)
+        assert math.isclose(LSE[0, 0, i], math.log(i + 1), rel_tol=1e-13, abs_tol=1e-15)
+
+
+def test_single_key_and_first_causal_row():
+    q, k, v = _rand(1, 1, 1, 4), _rand(1, 1, 1, 4), _rand(1, 1, 1, 4)
+    O, LSE = oracle.attention_forward(q, k, v, 0.5, False)
+    np.testing.assert_allclose(O[0, 0, 0], v[0, 0, 0], rtol=1e-15)
+    assert math.isclose(LSE[0, 0, 0], 0.5 * float(q[0, 0, 0] @ k[0, 0, 0]), rel_tol=1e-14)
+    q, k, v = _rand(1, 6, 1, 4), _rand(1, 6, 1, 4), _rand(1, 6, 1, 4)
+    O, LSE = oracle.attention_forward(q, k, v, 0.5, True)
+    np.testing.assert_allclose(O[0, 0, 0], v[0, 0, 0], rtol=1e-15)
+    assert math.isclose(LSE[0, 0, 0], 0.5 * float(q[0, 0, 0] @ k[0, 0, 0]), rel_tol=1e-14)
+
+
+def test_fully_masked_rows_are_zero():
+    """Causal with Tq > Tk: the first Tq-Tk rows see no key -> O=0, LSE=-inf, zero grads."""
+    Tq, Tk, d = 6, 3, 2
+    q, k, v, do = _rand(1, Tq, 1, d), _rand(1, Tk, 1, d), _rand(1, Tk, 1, d), _rand(1, Tq, 1, d)
+    O, LSE = oracle.attention_forward(q, k, v, 1.0, True)
+    assert np.all(O[0, :Tq - Tk] == 0) and np.all(np.isneginf(LSE[0, 0, :Tq - Tk]))
+    assert np.all(np.isfinite(LSE[0, 0, Tq - Tk:]))
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, 1.0, True)
+    assert np.all(dq[0, :Tq - Tk] == 0)
+    # Tk == 0
+    O, LSE = oracle.attention_forward(q, k[:, :0], v[:, :0], 1.0, False)
+    assert np.all(O == 0) and np.all(np.isneginf(LSE))
+
+
+def test_key_permutation_and_shift_invariance():
+    B, T, H, d = 1, 10, 1, 5
+    q, k, v, do = _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d)
+    s = 0.4
+    O, LSE = oracle.attention_forward(q, k, v, s, False)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, s, False)
+    perm = RNG.permutation(T)
+    O2, LSE2 = oracle.attention_forward(q, k[:, perm], v[:, perm], s, False)
+    dq2, dk2, dv2 = oracle.attention_backward(q, k[:, perm], v[:, perm], do, s, False)
+    np.testing.assert_allclose(O2, O, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(LSE2, LSE, rtol=1e-13)
+    np.testing.assert_allclose(dq2, dq, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dk2, dk[:, perm], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dv2, dv[:, perm], rtol=1e-11, atol=1e-12)
+    # shift: K + w leaves O unchanged and shifts LSE_i by s q_i . w
+    w = _rand(d)
+    O3, LSE3 = oracle.attention_forward(q, k + w, v, s, False)
+    np.testing.assert_allclose(O3, O, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(LSE3[0, 0], LSE[0, 0] + s * (q[0, :, 0] @ w), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Backward: finite differences, dK column sums, library cross-check, GQA
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_finite_differences(causal):
+    B, T, H, d = 1, 6, 1, 3
+    q, k, v, do = _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d)
+    s = 0.6
+
+    def loss(q_, k_, v_):
+        return float((oracle.attention_forward(q_, k_, v_, s, causal)[0] * do).sum())
+
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, s, causal)
+    eps = 1e-5
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            num[idx] = (loss(**{a + "_": b for a, b in args_p.items()})
+                        - loss(**{a + "_": b for a, b in args_m.items()})) / (2 * eps)
+        rel = np.linalg.norm(num - g) / np.linalg.norm(g)
+        assert rel <= 1e-6, (name, rel)
+
+
+def test_dk_columns_sum_to_zero():
+    """Each dS row sums to zero, so sum_j dK_j = 0 for every KV head."""
+    B, T, Hq, Hkv, d = 2, 8, 4, 2, 3
+    q, do = _rand(B, T, Hq, d), _rand(B, T, Hq, d)
+    k, v = _rand(B, T, Hkv, d), _rand(B, T, Hkv, d)
+    for causal in (False, True):
+        _, dk, _ = oracle.attention_backward(q, k, v, do, 0.5, causal)
+        np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_matches_torch_float64_sdpa(causal):
+    """Library special case: PyTorch's math SDPA + autograd in float64."""
+    B, T, H, d = 2, 7, 3, 4
+    q, k, v, do = _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d)
+    s = 0.45
+    O, LSE = oracle.attention_forward(q, k, v, s, causal)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, s, causal)
+    tq, tk, tv = (torch.tensor(x.transpose(0, 2, 1, 3), requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=s)
+    to.backward(torch.tensor(do.transpose(0, 2, 1, 3)))
+    np.testing.assert_allclose(O, to.detach().numpy().transpose(0, 2, 1, 3), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dq, tq.grad.numpy().transpose(0, 2, 1, 3), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy().transpose(0, 2, 1, 3), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy().transpose(0, 2, 1, 3), rtol=1e-10, atol=1e-11)
+    # LSE from the library's own logsumexp of the masked scaled scores
+    S = torch.tensor(q.transpose(0, 2, 1, 3)) @ torch.tensor(k.transpose(0, 2, 3, 1)) * s
+    if causal:
+        S = S.masked_fill(torch.ones(T, T, dtype=torch.bool).triu(1), float("-inf"))
+    np.testing.assert_allclose(LSE, torch.logsumexp(S, dim=-1).numpy(), rtol=1e-13)
+
+
+def test_gqa_equals_repeated_heads():
+    B, T, Hq, Hkv, d = 1, 6, 6, 2, 3
+    G = Hq // Hkv
+    q, do = _rand(B, T, Hq, d), _rand(B, T, Hq, d)
+    k, v = _rand(B, T, Hkv, d), _rand(B, T, Hkv, d)
+    krep, vrep = np.repeat(k, G, axis=2), np.repeat(v, G, axis=2)
+    for causal in (False, True):
+        O, LSE = oracle.attention_forward(q, k, v, 0.5, causal)
+        Or, LSEr = oracle.attention_forward(q, krep, vrep, 0.5, causal)
+        np.testing.assert_array_equal(O, Or)
+        np.testing.assert_array_equal(LSE, LSEr)
+        dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.5, causal)
+        dqr, dkr, dvr = oracle.attention_backward(q, krep, vrep, do, 0.5, causal)
+        np.testing.assert_allclose(dq, dqr, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(dk, dkr.reshape(B, T, Hkv, G, d).sum(3), rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(dv, dvr.reshape(B, T, Hkv, G, d).sum(3), rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Decode and the split-KV combine
+# ---------------------------------------------------------------------------
+
+def test_split_kv_any_chunk_size():
+    n, d = 300, 4
+    q = _rand(d)
+    kk, vv = _rand(n, d), _rand(n, d)
+    s = 0.5
+    o_ref, lse_ref = oracle.head_forward(q[None], kk, vv, s, False)
+    for chunk in (1, 7, 256, n):
+        parts_o, parts_l = [], []
+        for c0 in range(0, n, chunk):
+            o, l = oracle.head_forward(q[None], kk[c0:c0 + chunk], vv[c0:c0 + chunk], s, False)
+            parts_o.append(o[0])
+            parts_l.append(l[0])
+        o, lse = oracle.combine_partials(parts_o, parts_l)
+        np.testing.assert_allclose(o, o_ref[0], rtol=1e-12, atol=1e-13)
+        assert math.isclose(lse, lse_ref[0], rel_tol=1e-13)
+
+
+def test_combine_reproduces_two_tile_example():
+    g = read_golden("two_tile_example.txt")
+    sc, vals = g["scores"], g["values"]
+    parts = [oracle.brute_force_row(sc[i:i + 2], vals[i:i + 2]) for i in (0, 2)]
+    o, lse = oracle.combine_partials([[p[0]] for p in parts], [p[1] for p in parts])
+    l2 = math.exp(-1) * (1 + math.exp(-1)) + 1 + math.exp(-3)
+    u2 = math.exp(-1) * (10 + 20 * math.exp(-1)) + 30 + 40 * math.exp(-3)
+    assert math.isclose(o[0], u2 / l2, rel_tol=1e-12)
+    assert math.isclose(lse, 3.0 + math.log(l2), rel_tol=1e-14)
+
+
+def test_decode_is_prefill_row_over_prefix():
+    B, Hq, Hkv, d, Tmax = 3, 4, 2, 5, 40
+    q = _rand(B, Hq, d)
+    kc, vc = _rand(B, Tmax, Hkv, d), _rand(B, Tmax, Hkv, d)
+    seqlens = [1, 17, 40]
+    O, LSE = oracle.decode_forward(q, kc, vc, seqlens, 0.3)
+    for b in range(B):
+        n = seqlens[b]
+        # garbage beyond the prefix must not matter
+        kc2, vc2 = kc.copy(), vc.copy()
+        kc2[b, n:] = 1e3
+        vc2[b, n:] = -1e3
+        O2, LSE2 = oracle.decode_forward(q, kc2, vc2, seqlens, 0.3)
+        np.testing.assert_array_equal(O2[b], O[b])
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            Ob, Lb = oracle.attention_forward(q[b, h][None, None, None], kc[b, :n, g][None, :, None],
+                                              vc[b, :n, g][None, :, None], 0.3, False)
+            np.testing.assert_allclose(O[b, h], Ob[0, 0, 0], rtol=1e-13, atol=1e-14)
+            assert math.isclose(LSE[b, h], Lb[0, 0, 0], rel_tol=1e-14)
+    np.testing.assert_allclose(O[0], np.repeat(vc[0, 0], Hq // Hkv, axis=0), rtol=1e-15)
+
+
+def test_row_panels_do_not_change_results():
+    """Rows are processed in panels; a long causal head must equal the
+    brute-force row for rows in different panels."""
+    T, d = 2100, 2
+    q, k, v = _rand(T, d), _rand(T, d), _rand(T, d)
+    O, LSE = oracle.head_forward(q, k, v, 0.5, True)
+    for i in (0, 1, 2047, 2048, 2099):
+        scores = list(0.5 * (k[:i + 1] @ q[i]))
+        o0, l0 = oracle.brute_force_row(scores, list(v[:i + 1, 0]))
+        assert math.isclose(O[i, 0], o0, rel_tol=1e-11, abs_tol=1e-12)
+        assert math.isclose(LSE[i], l0, rel_tol=1e-12)
+    Os, Ls = oracle.head_forward(q, k, v, 0.5, True, rows=[5, 2099, 3000 - 1000])
+    np.testing.assert_array_equal(Os[1], O[2099])
+    np.testing.assert_array_equal(Ls[2], LSE[2000])

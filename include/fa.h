@@ -1,0 +1,155 @@
+/*
+ * fa.h -- C ABI of libfa: exact, IO-aware scaled-dot-product attention for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (all entry points compute the same function):
+ *   S = scale * Q K^T (+ causal mask), P = softmax(S) row by row, O = P V,
+ *   LSE_i = ln sum_j exp(S_ij).
+ * It is computed tile by tile with the online softmax, never writing S or P
+ * to device memory.  Sources, cited by page title and section:
+ *   - "Flash Attention: Why Memory Traffic, Not Compute, Is the Bottleneck",
+ *     sections "Flash Attention Uses Tiles", "Softmax Looks Like an Obstacle",
+ *     "Causal Masks Still Apply", "We Usually Call It Through an API";
+ *   - "Efficient attention: memory-bound", sections "Standard attention,
+ *     kernel by kernel" and "Real code moves even more" (the backward
+ *     products), "The obstacle, a normalizer that needs the whole row";
+ *   - "FlashAttention" (interview track), sections "Softmax without seeing
+ *     the whole row" (one fp32 log-sum-exp per row kept for the backward
+ *     pass, recomputation instead of storing P) and "In practice" (GQA,
+ *     causal masks, FlashDecoding's split of the KV cache).
+ *
+ * Conventions shared by every entry point
+ *   - Element types: bf16 = IEEE bfloat16 stored as uint16_t bit patterns;
+ *     float = IEEE fp32.  Accumulation is fp32.
+ *   - Layouts are dense, row-major "BTHD":
+ *       q, o, dO, dq   : [B, Tq, Hq, d]
+ *       k, v, dk, dv   : [B, Tk, Hkv, d]
+ *       lse            : [B, Hq, Tq]   (natural-log units of the scaled scores)
+ *   - d must be 64 or 128; Hq % Hkv == 0.  Query head h reads KV head
+ *     h / (Hq / Hkv) (contiguous groups).
+ *   - Causal rule: key j is visible to query i iff j <= i + (Tk - Tq)
+ *     (bottom-right aligned; for Tq == Tk this is j <= i).  A row that sees
+ *     no key gets O = 0, LSE = -inf and zero gradients.
+ *   - All pointers are DEVICE pointers of the current CUDA device, 16-byte
+ *     aligned.  The caller owns every buffer, including workspaces; the
+ *     library never allocates or frees device memory (except where an entry
+ *     point says otherwise).
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t passed
+ *     as void*; NULL = legacy default stream).  Nothing synchronises.
+ *   - Inputs are never modified.
+ *   - Return value: FA_OK or one of the fa_status codes.  Argument errors are
+ *     detected on the host before anything is launched.  A kernel whose
+ *     bounded wait expires records FA_ERR_TIMEOUT in a device status word,
+ *     which fa_check() reports.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* bad size, null pointer, Hq % Hkv != 0, ... */
+  FA_ERR_UNSUPPORTED = 2,  /* head dim other than 64/128, device not sm_100 */
+  FA_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = 4,    /* workspace pointer null or smaller than required */
+  FA_ERR_CUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
+  FA_ERR_TIMEOUT = 6       /* a kernel's bounded wait expired (see fa_check) */
+} fa_status;
+
+/* Human-readable name of a status code (static string). */
+const char* fa_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int fa_version(void);
+
+/*
+ * fa_forward -- O and LSE of exact attention.
+ * ("Flash Attention: Why Memory Traffic...", "Flash Attention Uses Tiles" and
+ *  "Softmax Looks Like an Obstacle"; LSE as in "FlashAttention",
+ *  "Softmax without seeing the whole row".)
+ *   q [B,Tq,Hq,d], k/v [B,Tk,Hkv,d]  bf16 in
+ *   o [B,Tq,Hq,d] bf16 out; lse [B,Hq,Tq] fp32 out
+ *   scale: multiplies QK^T before the softmax (usually 1/sqrt(d))
+ *   causal: 0 or 1
+ * Tq == 0 is a no-op.  Tk == 0 writes O = 0 and LSE = -inf.
+ */
+int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
+               int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal,
+               void* stream);
+
+/*
+ * Bytes of device workspace fa_backward needs: an fp32 dQ accumulator
+ * [B,Tq,Hq,d] plus the fp32 row terms D_i = sum_c dO_ic O_ic [B,Hq,Tq],
+ * rounded up to 256-byte pieces.
+ */
+size_t fa_backward_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int d);
+
+/*
+ * fa_backward -- dQ, dK, dV of L = sum(dO * O) for the forward above, with
+ * S and P recomputed tile by tile from the saved LSE ("FlashAttention",
+ * follow-up on recomputing instead of storing P; the products dV = P^T dO,
+ * dP = dO V^T, dS = P*(dP - D), dQ = scale dS K, dK = scale dS^T Q from
+ * "Efficient attention: memory-bound", "Real code moves even more").
+ *   q, k, v, o (the forward's output), lse (the forward's LSE), dO  in
+ *   dq [B,Tq,Hq,d], dk/dv [B,Tk,Hkv,d] bf16 out.  For GQA, dk/dv sum over the
+ *   query heads of each group.
+ *   ws/ws_bytes: device workspace of at least fa_backward_workspace_bytes();
+ *   its contents on entry do not matter.
+ */
+int fa_backward(const void* q, const void* k, const void* v, const void* o,
+                const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                void* ws, size_t ws_bytes,
+                int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal,
+                void* stream);
+
+/*
+ * Bytes of device workspace fa_decode_splitkv needs: fp32 partial outputs
+ * [B,Hq,nchunk,d] and partial LSEs [B,Hq,nchunk], nchunk = ceil(Tk_max/chunk).
+ */
+size_t fa_decode_workspace_bytes(int B, int Hq, int Tk_max, int d, int chunk);
+
+/*
+ * fa_decode_splitkv -- one query token per sequence against a KV cache,
+ * split into chunks of `chunk` keys processed by separate thread blocks and
+ * merged by their log-sum-exp ("FlashAttention", "In practice":
+ * FlashDecoding).
+ *   q [B,Hq,d] bf16; k_cache/v_cache [B,Tk_max,Hkv,d] bf16;
+ *   seqlens_k: DEVICE int32 [B], each in [0, Tk_max] (sequence b attends to
+ *   its first seqlens_k[b] cached keys, no mask);
+ *   o [B,Hq,d] bf16 out; lse [B,Hq] fp32 out;
+ *   ws/ws_bytes: at least fa_decode_workspace_bytes(); contents on entry do
+ *   not matter.  chunk must be a positive multiple of 64.
+ *   Hq/Hkv must be 1, 2, 4 or 8 and chunk * (Hq/Hkv) at most 4096.
+ */
+int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                      const int* seqlens_k, void* o, float* lse, void* ws, size_t ws_bytes,
+                      int B, int Hq, int Hkv, int Tk_max, int d, float scale, int chunk,
+                      void* stream);
+
+/*
+ * fa_check -- synchronise `stream`, then read and clear the device status
+ * word that kernels set when a bounded wait expires.  Returns FA_OK,
+ * FA_ERR_TIMEOUT, or FA_ERR_CUDA if the synchronisation itself failed.
+ */
+int fa_check(void* stream);
+
+/*
+ * fa_selftest_bounded_wait -- launch one block that waits on a barrier that
+ * nothing will ever complete, with a wait limit of `limit_us` microseconds
+ * (1..1000000).  The kernel gives up, records FA_ERR_TIMEOUT in the status
+ * word and returns normally; fa_check() then reports it.  Used to test the
+ * failure path without faulting or hanging the GPU.
+ */
+int fa_selftest_bounded_wait(int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,20 @@
+"""io_aware_exact_forward_b200 -- exact IO-aware attention for B200 (sm_100a).
+
+The computation lives in libfa.so (hand-written CUDA kernels behind the C ABI
+of include/fa.h); this package only marshals torch tensors into that ABI.
+"""
+
+from ._binding import (  # noqa: F401
+    FAError,
+    LIB_PATH,
+    SIGNATURES,
+    STATUS,
+    backward,
+    backward_workspace_bytes,
+    check,
+    decode_splitkv,
+    decode_workspace_bytes,
+    forward,
+    load_library,
+    selftest_bounded_wait,
+)

@@ -1,0 +1,182 @@
+"""ctypes binding of libfa (include/fa.h).
+
+Argument marshalling only: every step of the attention computation runs in
+the CUDA kernels of libfa.so.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+STATUS = {
+    0: "FA_OK",
+    1: "FA_ERR_INVALID_ARG",
+    2: "FA_ERR_UNSUPPORTED",
+    3: "FA_ERR_ALIGNMENT",
+    4: "FA_ERR_WORKSPACE",
+    5: "FA_ERR_CUDA",
+    6: "FA_ERR_TIMEOUT",
+}
+
+# Every symbol include/fa.h declares, with its ctypes signature.
+_c_int, _c_float, _c_size, _vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+SIGNATURES = {
+    "fa_status_string": (ctypes.c_char_p, [_c_int]),
+    "fa_version": (_c_int, []),
+    "fa_forward": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_backward_workspace_bytes": (_c_size, [_c_int] * 6),
+    "fa_backward": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_decode_workspace_bytes": (_c_size, [_c_int] * 5),
+    "fa_decode_splitkv": (_c_int, [_vp] * 6 + [_vp, _c_size] + [_c_int] * 5 + [_c_float, _c_int, _vp]),
+    "fa_check": (_c_int, [_vp]),
+    "fa_selftest_bounded_wait": (_c_int, [_c_int, _vp]),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfa.so (built in-tree by io_aware_exact_forward_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(
+                f"libfa.so not found at {path}; build it with "
+                "`python -m io_aware_exact_forward_b200.build` (no CPU fallback exists)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _stream_ptr(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check_dev(name, t, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (libfa has no CPU path)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _raise(fn, st):
+    if st != 0:
+        raise FAError(fn, st)
+
+
+def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
+    """O, LSE = attention(q, k, v).  q [B,Tq,Hq,d], k/v [B,Tk,Hkv,d] bf16 (CUDA)."""
+    lib = load_library()
+    B, Tq, Hq, d = q.shape
+    Tk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_dev(n, t, torch.bfloat16, dev)
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=dev)
+    _check_dev("out", out, torch.bfloat16, dev)
+    _check_dev("lse", lse, torch.float32, dev)
+    st = lib.fa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tk, d,
+                        float(scale), int(bool(causal)), _stream_ptr(dev))
+    _raise("fa_forward", st)
+    return out, lse
+
+
+def backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d) -> int:
+    return int(load_library().fa_backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d))
+
+
+def backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV for L = sum(dO * O).  `workspace` (uint8 CUDA tensor) is
+    allocated here when not given."""
+    lib = load_library()
+    B, Tq, Hq, d = q.shape
+    Tk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_dev(n, t, torch.bfloat16, dev)
+    _check_dev("lse", lse, torch.float32, dev)
+    if scale is None:
+        scale = d ** -0.5
+    need = backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib.fa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                         _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tq, Tk, d,
+                         float(scale), int(bool(causal)), _stream_ptr(dev))
+    _raise("fa_backward", st)
+    return dq, dk, dv
+
+
+def decode_workspace_bytes(B, Hq, Tk_max, d, chunk=256) -> int:
+    return int(load_library().fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk))
+
+
+def decode_splitkv(q, k_cache, v_cache, seqlens, scale=None, chunk=256, workspace=None, out=None, lse=None):
+    """Split-KV decode.  q [B,Hq,d], caches [B,Tk_max,Hkv,d] bf16, seqlens int32 [B] (CUDA)."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    Tk_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+    dev = q.device
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_dev(n, t, torch.bfloat16, dev)
+    _check_dev("seqlens", seqlens, torch.int32, dev)
+    if scale is None:
+        scale = d ** -0.5
+    need = decode_workspace_bytes(B, Hq, Tk_max, d, chunk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev) if lse is None else lse
+    st = lib.fa_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse),
+                               _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tk_max, d, float(scale),
+                               int(chunk), _stream_ptr(dev))
+    _raise("fa_decode_splitkv", st)
+    return out, lse
+
+
+def check(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    return int(load_library().fa_check(_stream_ptr(dev)))
+
+
+def selftest_bounded_wait(limit_us: int, device=None) -> int:
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    return int(load_library().fa_selftest_bounded_wait(int(limit_us), _stream_ptr(dev)))

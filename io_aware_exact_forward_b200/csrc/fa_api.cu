@@ -1,0 +1,332 @@
+// fa_api.cu -- the C ABI of libfa (declared in include/fa.h): argument
+// checks, TMA descriptor set-up and kernel launches.  Every kernel of the
+// library is compiled in this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "fa_status.h"
+#include "fa_ptx.cuh"
+#include "fa_fwd.cuh"
+#include "fa_bwd.cuh"
+#include "fa_decode.cuh"
+
+namespace fa {
+
+// Limit for every bounded wait inside the kernels.  Far above any legitimate
+// wait (the longest kernels run for tens of milliseconds).
+static constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+
+// ---------------------------------------------------------------------------
+// Driver entry point for TMA descriptors (resolved through the runtime, so
+// the library links no driver stub and loads on machines without a GPU).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor [n3][n2][n1][n0] (n0 contiguous) with box {64, 1, box_rows, 1}
+// along (n0, n1, n2, n3) and the 128-byte swizzle, or no swizzle when
+// `swizzle` is false (then box_inner elements along n0).
+static int make_tmap_4d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
+                        uint64_t n3, uint32_t box_inner, uint32_t box_rows, bool swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {n0, n1, n2, n3};
+  const cuuint64_t strides[3] = {n0 * 2, n0 * n1 * 2, n0 * n1 * n2 * 2};
+  const cuuint32_t box[4] = {box_inner, 1, box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Per-device set-up: architecture check and shared-memory opt-in, once.
+// ---------------------------------------------------------------------------
+static constexpr int kMaxDevices = 64;
+
+template <typename Fn>
+static int set_smem(Fn* kernel, int bytes) {
+  return cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel),
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
+template <int D, int G>
+static int decode_setup_one() {
+  int st = set_smem(fa_decode_split_kernel<D, G>, DecCfg<D, G>::SMEM_BYTES);
+  return st;
+}
+
+static int decode_setup() {
+  int st = FA_OK;
+  if (!st) st = decode_setup_one<64, 1>();
+  if (!st) st = decode_setup_one<64, 2>();
+  if (!st) st = decode_setup_one<64, 4>();
+  if (!st) st = decode_setup_one<64, 8>();
+  if (!st) st = decode_setup_one<128, 1>();
+  if (!st) st = decode_setup_one<128, 2>();
+  if (!st) st = decode_setup_one<128, 4>();
+  if (!st) st = decode_setup_one<128, 8>();
+  return st;
+}
+
+static int device_setup_impl() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
+  int st = FA_OK;
+  if (!st) st = set_smem(fa_fwd_kernel<64>, FwdCfg<64>::SMEM_BYTES);
+  if (!st) st = set_smem(fa_fwd_kernel<128>, FwdCfg<128>::SMEM_BYTES);
+  if (!st) st = bwd_setup();
+  if (!st) st = decode_setup();
+  return st;
+}
+
+static int device_setup() {
+  static int state[kMaxDevices];  // 0 = not done, else status + 1
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (state[dev] == 0) state[dev] = device_setup_impl() + 1;
+  return state[dev] - 1;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Checks shared by the prefill entry points.
+static int check_prefill(int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Tq < 0 || Tk < 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // Tensor-map extents are 32-bit and row indices are int.
+  if ((int64_t)Tq > (1 << 30) || (int64_t)Tk > (1 << 30) || (int64_t)B * Hq > (1 << 30))
+    return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_version(void) { return 100; }
+
+int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Tq, int Tk, int d, float scale, int causal, void* stream) {
+  int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
+  if (st) return st;
+  if (B == 0 || Tq == 0) return FA_OK;
+  if (!q || !o || !lse || (Tk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || (Tk > 0 && (!aligned16(k) || !aligned16(v))))
+    return FA_ERR_ALIGNMENT;
+  st = device_setup();
+  if (st) return st;
+  FwdParams p;
+  memset(&p, 0, sizeof(p));
+  st = make_tmap_4d(&p.tm_q, q, d, Hq, Tq, B, 64, 128, true);
+  if (!st && Tk > 0) st = make_tmap_4d(&p.tm_k, k, d, Hkv, Tk, B, 64, 128, true);
+  if (!st && Tk > 0) st = make_tmap_4d(&p.tm_v, v, d, Hkv, Tk, B, 64, 128, true);
+  if (st) return st;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tq = Tq; p.Tk = Tk;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_mblocks = (Tq + 255) / 256;
+  p.wait_limit_ns = kWaitLimitNs;
+  dim3 grid(B * Hq, p.n_mblocks);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    fa_fwd_kernel<64><<<grid, FwdCfg<64>::THREADS, FwdCfg<64>::SMEM_BYTES, s>>>(p);
+  else
+    fa_fwd_kernel<128><<<grid, FwdCfg<128>::THREADS, FwdCfg<128>::SMEM_BYTES, s>>>(p);
+  return launch_status();
+}
+
+size_t fa_backward_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int d) {
+  (void)Hkv; (void)Tk;
+  if (B < 0 || Hq < 1 || Tq < 0 || (d != 64 && d != 128)) return 0;
+  const size_t dq = ((size_t)B * Tq * Hq * d * 4 + 255) / 256 * 256;
+  const size_t dd = ((size_t)B * Hq * Tq * 4 + 255) / 256 * 256;
+  return dq + dd;
+}
+
+int fa_backward(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B,
+                int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal, void* stream) {
+  int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
+  if (st) return st;
+  if (B == 0 || (Tq == 0 && Tk == 0)) return FA_OK;
+  if ((Tq > 0 && (!q || !o || !lse || !dO || !dq)) || (Tk > 0 && (!k || !v || !dk || !dv)))
+    return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return FA_ERR_ALIGNMENT;
+  const size_t need = fa_backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return FA_ERR_WORKSPACE;
+  (void)stream;
+  return FA_ERR_UNSUPPORTED;
+}
+
+static size_t decode_nchunk(int Tk_max, int chunk) { return ((size_t)Tk_max + chunk - 1) / chunk; }
+
+size_t fa_decode_workspace_bytes(int B, int Hq, int Tk_max, int d, int chunk) {
+  if (B < 0 || Hq < 1 || Tk_max < 0 || chunk < 1 || (d != 64 && d != 128)) return 0;
+  const size_t n = decode_nchunk(Tk_max, chunk);
+  const size_t wo = ((size_t)B * Hq * n * d * 4 + 255) / 256 * 256;
+  const size_t wl = ((size_t)B * Hq * n * 4 + 255) / 256 * 256;
+  return wo + wl;
+}
+
+int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
+                      void* o, float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv,
+                      int Tk_max, int d, float scale, int chunk, void* stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Tk_max < 0 || Hq % Hkv != 0 || !isfinite(scale))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
+  if (chunk < 64 || chunk % 64 != 0 || chunk * G > 4096) return FA_ERR_INVALID_ARG;
+  if ((int64_t)Tk_max > (1 << 30) || (int64_t)B * Hq > (1 << 30)) return FA_ERR_INVALID_ARG;
+  if (B == 0) return FA_OK;
+  if (!q || !seqlens_k || !o || !lse || (Tk_max > 0 && (!k_cache || !v_cache)))
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) ||
+      (Tk_max > 0 && (!aligned16(k_cache) || !aligned16(v_cache))))
+    return FA_ERR_ALIGNMENT;
+  const size_t need = fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return FA_ERR_WORKSPACE;
+  int st = device_setup();
+  if (st) return st;
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  const size_t n = decode_nchunk(Tk_max, chunk);
+  if (Tk_max > 0) {
+    st = make_tmap_4d(&p.tm_k, k_cache, d, Hkv, Tk_max, B, d, 64, false);
+    if (!st) st = make_tmap_4d(&p.tm_v, v_cache, d, Hkv, Tk_max, B, d, 64, false);
+    if (st) return st;
+  }
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.seqlens = seqlens_k;
+  p.ws_o = reinterpret_cast<float*>(ws);
+  p.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) +
+                                      ((size_t)B * Hq * n * d * 4 + 255) / 256 * 256);
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tk_max = Tk_max; p.chunk = chunk; p.nchunk = (int)n;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = kWaitLimitNs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (Tk_max > 0) {
+    dim3 grid((unsigned)n, Hkv, B);
+#define FA_DEC_LAUNCH(DD, GG) \
+    fa_decode_split_kernel<DD, GG><<<grid, DecCfg<DD, GG>::THREADS, DecCfg<DD, GG>::SMEM_BYTES, s>>>(p)
+    if (d == 64) {
+      if (G == 1) FA_DEC_LAUNCH(64, 1); else if (G == 2) FA_DEC_LAUNCH(64, 2);
+      else if (G == 4) FA_DEC_LAUNCH(64, 4); else FA_DEC_LAUNCH(64, 8);
+    } else {
+      if (G == 1) FA_DEC_LAUNCH(128, 1); else if (G == 2) FA_DEC_LAUNCH(128, 2);
+      else if (G == 4) FA_DEC_LAUNCH(128, 4); else FA_DEC_LAUNCH(128, 8);
+    }
+#undef FA_DEC_LAUNCH
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  const int warps = B * Hq;
+  const int blocks = (warps * 32 + 255) / 256;
+  if (d == 64)
+    fa_decode_combine_kernel<64><<<blocks, 256, 0, s>>>(p);
+  else
+    fa_decode_combine_kernel<128><<<blocks, 256, 0, s>>>(p);
+  return launch_status();
+}
+
+int fa_check(void* stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"
+
+namespace fa {
+// One block, one thread waits on a barrier that nothing completes.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtl w{&abort_flag, limit_ns};
+    mbar_wait(smem_u32(&bar), 0, w);
+  }
+  __syncthreads();
+}
+}  // namespace fa
+
+extern "C" int fa_selftest_bounded_wait(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return FA_ERR_INVALID_ARG;
+  int st = device_setup();
+  if (st) return st;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)limit_us * 1000ull);
+  return launch_status();
+}

@@ -1,0 +1,101 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every symbol include/fa.h declares, and rejects bad arguments before any
+launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import io_aware_exact_forward_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = _header_functions()
+    for n in ("fa_forward", "fa_backward", "fa_decode_splitkv", "fa_backward_workspace_bytes",
+              "fa_decode_workspace_bytes", "fa_check", "fa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = fa.load_library()
+    for n in _header_functions():
+        assert hasattr(lib, n), n
+        assert n in fa.SIGNATURES, f"binding lacks a signature for {n}"
+
+
+def test_status_strings():
+    lib = fa.load_library()
+    for code, name in fa.STATUS.items():
+        assert lib.fa_status_string(code).decode() == name
+
+
+NULL = None
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (B, Hq, Hkv, Tq, Tk, d, scale, causal)
+    ((1, 1, 1, 16, 16, 96, 1.0, 0), 2),      # unsupported head dim
+    ((1, 3, 2, 16, 16, 64, 1.0, 0), 1),      # Hq % Hkv != 0
+    ((1, 1, 1, 16, 16, 64, 1.0, 2), 1),      # causal not 0/1
+    ((1, 1, 1, -1, 16, 64, 1.0, 0), 1),      # negative length
+    ((1, 1, 1, 16, 16, 64, float("nan"), 0), 1),
+    ((1, 1, 1, 16, 16, 64, 1.0, 0), 1),      # null pointers
+    ((0, 1, 1, 16, 16, 64, 1.0, 0), 0),      # empty batch: no-op
+    ((1, 1, 1, 0, 16, 64, 1.0, 0), 0),       # empty query: no-op
+])
+def test_forward_rejects_bad_arguments_on_host(args, expect):
+    lib = fa.load_library()
+    assert lib.fa_forward(NULL, NULL, NULL, NULL, NULL, *args, NULL) == expect
+
+
+def test_forward_alignment_checked_before_launch():
+    lib = fa.load_library()
+    buf = (ctypes.c_uint8 * 64)()
+    base = ctypes.addressof(buf)
+    odd = ctypes.c_void_p(base + (16 - base % 16) + 2)
+    st = lib.fa_forward(odd, odd, odd, odd, odd, 1, 1, 1, 16, 16, 64, 1.0, 0, NULL)
+    assert st == 3
+
+
+def test_backward_and_decode_argument_checks():
+    lib = fa.load_library()
+    assert lib.fa_backward(*([NULL] * 9), NULL, 0, 1, 1, 1, 16, 16, 80, 1.0, 0, NULL) == 2
+    assert lib.fa_backward(*([NULL] * 9), NULL, 0, 1, 2, 3, 16, 16, 64, 1.0, 0, NULL) == 1
+    # decode: G must be 1,2,4,8; chunk a multiple of 64; chunk*G <= 4096
+    assert lib.fa_decode_splitkv(*([NULL] * 6), NULL, 0, 2, 32, 2, 1024, 128, 0.1, 256, NULL) == 2
+    assert lib.fa_decode_splitkv(*([NULL] * 6), NULL, 0, 2, 32, 8, 1024, 128, 0.1, 100, NULL) == 1
+    assert lib.fa_decode_splitkv(*([NULL] * 6), NULL, 0, 2, 32, 4, 1024, 128, 0.1, 2048, NULL) == 1
+    assert lib.fa_decode_splitkv(*([NULL] * 6), NULL, 0, 2, 32, 8, 1024, 128, 0.1, 256, NULL) == 1
+
+
+def test_workspace_sizes():
+    lib = fa.load_library()
+    B, Hq, T, d = 2, 4, 100, 64
+    ws = lib.fa_backward_workspace_bytes(B, Hq, 2, T, T, d)
+    assert ws >= B * T * Hq * d * 4 + B * Hq * T * 4
+    assert ws % 256 == 0
+    dws = lib.fa_decode_workspace_bytes(64, 32, 32768, 128, 256)
+    n = 32768 // 256
+    assert dws >= 64 * 32 * n * (128 + 1) * 4
+    assert lib.fa_decode_workspace_bytes(1, 1, 10, 96, 256) == 0
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The package must never import or call the CPU oracle."""
+    pkg = os.path.join(ROOT, "io_aware_exact_forward_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower() or f.endswith((".cu", ".cuh", ".h")) and "oracle" not in text, f
+                assert "import oracle" not in text and "from oracle" not in text, f

@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark: exact attention forward + backward on B200 through libfa.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa|reference]
+                    [--workload 2] [--no-e2e] [--no-cpu-baseline]
+
+One step = fa_forward + the three backward steps (preprocess, dK/dV, dQ
+finalize) over one batch of the GPT-2-medium-shaped layer (B=64, H=16,
+T=1024, d=64, non-causal; the workload the "Efficient attention: memory-bound"
+page times), bf16 inputs already resident in HBM.  Each step's inputs
+(4 x 128 MiB) exceed the 126 MB L2, so no flush is needed between steps.
+
+Prints one JSON line (rank 0).  `value` is algorithmic TFLOP/s of the whole
+job: (4 + 10) * B * Hq * d * pairs per step and GPU, over the slowest rank's
+device time.  Under torchrun each rank runs its own batch (the (batch, head)
+units are independent; no collective on the data path): weak scaling.
+
+`--impl reference` times the CPU float64 oracle (the reference arm here) on a
+bounded sample per step, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd+bwd TFLOPS (bf16, 1×B200) and % of dense tensor peak"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["fa", "reference"], default="fa")
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def pairs_count(Tq, Tk, causal):
+    """(query, key) pairs entering the softmax; bottom-right causal rule."""
+    if not causal:
+        return Tq * Tk
+    off = Tk - Tq
+    # rows i with i + off + 1 in [1, Tk]: sum of min(Tk, max(0, i + off + 1))
+    tot = 0
+    first_full = max(0, Tk - off - 1)   # from this row on every key is visible
+    for i in range(min(Tq, first_full)):
+        tot += max(0, i + off + 1)
+    tot += max(0, Tq - first_full) * Tk
+    return tot
+
+
+def flops(w):
+    P = pairs_count(w.T, w.T, w.causal)
+    f = 4 * w.B * w.Hq * w.d * P
+    b = 10 * w.B * w.Hq * w.d * P
+    return f, b
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"bf16_tflops": pk["bf16_tflops"], "bf16_tflops_sustained": pk.get("bf16_tflops_sustained"),
+                "hbm_gbs": pk["hbm_gbs"], "source": "measured"}
+    except Exception:
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "io_aware_exact_forward_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, only if it was
+    taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            data = json.load(f)
+        ent = data[kernel][workload]
+        if ent.get("source_hash") == kernel_source_hash():
+            return ent["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.out is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+                except ValueError:
+                    continue
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r[2] > 300.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3][1:5]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(load), "power_w_max": max(r[2] for r in rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_heads(w, inp_cpu, heads, budget_s):
+    """Run the oracle's forward + backward head by head; stop at the budget.
+    Returns (heads done, seconds, algorithmic flops done)."""
+    import oracle
+    from workloads import to_f64
+    G = w.Hq // w.Hkv
+    f, b = flops(w)
+    per_head = (f + b) / (w.B * w.Hq)
+    done, t0 = 0, time.perf_counter()
+    for (bi, h) in heads:
+        g = h // G
+        qh = to_f64(inp_cpu["q"][bi, :, h])
+        kh = to_f64(inp_cpu["k"][bi, :, g])
+        vh = to_f64(inp_cpu["v"][bi, :, g])
+        dh = to_f64(inp_cpu["do"][bi, :, h])
+        oracle.head_forward(qh, kh, vh, w.scale, w.causal)
+        oracle.head_backward(qh, kh, vh, dh, w.scale, w.causal)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done, dt, done * per_head
+
+
+def cpu_baseline(w, inp_cpu, budget_s):
+    heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    done, dt, fl = oracle_heads(w, inp_cpu, heads, budget_s)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"float64 oracle forward+backward of {done} of {w.B * w.Hq} heads of {w.name} "
+                      f"({dt:.1f} s; same algorithmic FLOP count as the GPU metric)"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm
+# ---------------------------------------------------------------------------
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return 0
+    from workloads import prefill_inputs
+    inp = prefill_inputs(w.with_(B=1), device="cpu")
+    heads = [(0, h) for h in range(w.Hq)]
+    for s in range(args.warmup):
+        oracle_heads(w, inp, [heads[s % len(heads)]], 1e9)
+    total_fl, total_t = 0.0, 0.0
+    for s in range(args.steps):
+        done, dt, fl = oracle_heads(w, inp, [heads[s % len(heads)]], 1e9)
+        total_fl += fl
+        total_t += dt
+    value = total_fl / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d,
+                   "causal": w.causal, "step": "one head of the workload, forward + backward"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one (batch, head) of {w.name} per step, float64 numpy"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# libfa arm
+# ---------------------------------------------------------------------------
+
+def run_fa(args, w, rank, world, dist):
+    import ctypes
+    import torch
+    import io_aware_exact_forward_b200 as fa
+    from workloads import prefill_inputs
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = fa.load_library()
+    inp = prefill_inputs(w, device=dev, seed=w.seed + rank)
+    q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
+    B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = lib.fa_backward_workspace_bytes(B, Hq, Hkv, T, T, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    P = ctypes.c_void_p
+    pq, pk, pv, pdo, po, plse = (P(t.data_ptr()) for t in (q, k, v, do, o, lse))
+    pdq, pdk, pdv, pws = (P(t.data_ptr()) for t in (dq, dk, dv, ws))
+    stream = torch.cuda.current_stream(dev)
+    sp = P(stream.cuda_stream)
+    scale, causal = w.scale, int(w.causal)
+
+    def check(st, name):
+        if st != 0:
+            raise RuntimeError(f"{name}: {fa.STATUS.get(st, st)}")
+
+    def step(evs=None):
+        if evs: evs[0].record(stream)
+        check(lib.fa_forward(pq, pk, pv, po, plse, B, Hq, Hkv, T, T, d, scale, causal, sp), "fa_forward")
+        if evs: evs[1].record(stream)
+        check(lib.fa_backward_preprocess(po, plse, pdo, pws, ws_bytes, B, Hq, Hkv, T, T, d, sp), "preprocess")
+        if evs: evs[2].record(stream)
+        check(lib.fa_backward_dkdv(pq, pk, pv, pdo, pdk, pdv, pws, ws_bytes, B, Hq, Hkv, T, T, d, scale, causal,
+                                   sp), "dkdv")
+        if evs: evs[3].record(stream)
+        check(lib.fa_backward_dq_finalize(pdq, pws, ws_bytes, B, Hq, Hkv, T, T, d, sp), "dq_finalize")
+        if evs: evs[4].record(stream)
+
+    kernels_per_step = 4
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if lib.fa_check(sp) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    gpu_index = local
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            gpu_index = int(vis.split(",")[local])
+        except ValueError:
+            pass
+    barrier()
+    with ClockSampler(gpu_index) as clocks:
+        t_start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t_end.record(stream)
+        barrier()
+    status = lib.fa_check(sp)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    elapsed_ms = t_start.elapsed_time(t_end)
+    seg = [sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps for i in range(4)]
+    if dist is not None:
+        import torch.distributed as tdist
+        t = torch.tensor([elapsed_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    f_fwd, f_bwd = flops(w)
+    value = world * (f_fwd + f_bwd) * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel (largest share of the step)
+    peaks = load_peaks()
+    names = ["fa_fwd_kernel", "fa_bwd_preprocess_kernel", "fa_bwd_dkdv_kernel", "fa_bwd_dq_convert_kernel"]
+    dom = max(range(4), key=lambda i: seg[i])
+    if dom == 0:
+        alg, bound = f_fwd, "tensor"
+    elif dom == 2:
+        alg, bound = f_bwd, "tensor"
+    else:
+        alg, bound = None, "hbm"
+    if alg is not None:
+        achieved = alg / (seg[dom] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"kernel": names[dom], "bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                "traffic": traffic_from_profile(names[dom], w.name), "traffic_unit": "bytes per launch",
+                "algorithmic_per_launch": alg}
+    else:
+        roof = {"kernel": names[dom], "bound": bound, "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": None, "traffic": None}
+    per_kernel = {names[i]: {"ms_avg": seg[i]} for i in range(4)}
+    per_kernel["fa_fwd_kernel"]["tflops"] = f_fwd / (seg[0] * 1e-3) / 1e12
+    per_kernel["fa_bwd_dkdv_kernel"]["tflops"] = f_bwd / (seg[2] * 1e-3) / 1e12
+    per_kernel["backward_total_tflops"] = f_bwd / (sum(seg[1:]) * 1e-3) / 1e12
+
+    # end to end through the public API, host buffers in pinned memory
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        hdq = torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True)
+        hdk = torch.empty(dk.shape, dtype=dk.dtype, pin_memory=True)
+        hdv = torch.empty(dv.shape, dtype=dv.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True); do.copy_(hdo, non_blocking=True)
+            fa.forward(q, k, v, scale=scale, causal=w.causal, out=o, lse=lse)
+            fa.backward(q, k, v, o, lse, do, scale=scale, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+            ho.copy_(o, non_blocking=True); hlse.copy_(lse, non_blocking=True)
+            hdq.copy_(dq, non_blocking=True); hdk.copy_(dk, non_blocking=True); hdv.copy_(dv, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            import torch.distributed as tdist
+            t = torch.tensor([e_ms], device=dev)
+            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * (f_fwd + f_bwd) * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "ms_per_step": e_ms / args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = {n: inp[n].cpu() for n in ("q", "k", "v", "do")}
+        cpu = cpu_baseline(w, inp_cpu, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
+                       "step": "fa_forward + fa_backward (preprocess, dkdv, dq_finalize)",
+                       "l2": "inputs larger than L2 (q, k, v, dO: 4 x %d MiB per step)" % (q.numel() * 2 >> 20),
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "seed": w.seed},
+            "pct_of_peak": {"measured": value / world / peaks["bf16_tflops"], "spec_2250": value / world / 2250.0},
+            "roofline": roof,
+            "per_kernel": per_kernel,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": kernels_per_step * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    from workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        return run_reference(args, w, rank)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        return run_fa(args, w, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -85,8 +85,9 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
 
 /*
  * Bytes of device workspace fa_backward needs: an fp32 dQ accumulator
- * [B,Tq,Hq,d] plus the fp32 row terms D_i = sum_c dO_ic O_ic [B,Hq,Tq],
- * rounded up to 256-byte pieces.
+ * [B,Tq,Hq,d], the fp32 row terms D_i = sum_c dO_ic O_ic [B,Hq,Tq] and the
+ * LSE in log2 units [B,Hq,Tq], each rounded up to 256 bytes.  Returns 0 for
+ * invalid sizes.
  */
 size_t fa_backward_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int d);
 
@@ -107,6 +108,27 @@ int fa_backward(const void* q, const void* k, const void* v, const void* o,
                 void* ws, size_t ws_bytes,
                 int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal,
                 void* stream);
+
+/*
+ * The three steps fa_backward runs, in this order on one stream, exposed so
+ * that a caller can schedule or time them separately.  They share the
+ * workspace of fa_backward_workspace_bytes() and its layout; arguments mean
+ * what they mean for fa_backward.
+ *   fa_backward_preprocess   D_i = sum_c dO_ic O_ic and the LSE in log2
+ *                            units into the workspace; zeroes the fp32 dQ
+ *                            accumulator.
+ *   fa_backward_dkdv         one pass over (key tile, KV head, batch): dK and
+ *                            dV written, scale*dS*K added into the dQ
+ *                            accumulator.  Needs the preprocess step first.
+ *   fa_backward_dq_finalize  dq = bf16(accumulator).
+ */
+int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void* ws, size_t ws_bytes,
+                           int B, int Hq, int Hkv, int Tq, int Tk, int d, void* stream);
+int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                     void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+                     float scale, int causal, void* stream);
+int fa_backward_dq_finalize(void* dq, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk,
+                            int d, void* stream);
 
 /*
  * Bytes of device workspace fa_decode_splitkv needs: fp32 partial outputs

@@ -34,6 +34,9 @@ SIGNATURES = {
     "fa_forward": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_workspace_bytes": (_c_size, [_c_int] * 6),
     "fa_backward": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_backward_preprocess": (_c_int, [_vp] * 4 + [_c_size] + [_c_int] * 6 + [_vp]),
+    "fa_backward_dkdv": (_c_int, [_vp] * 7 + [_c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_backward_dq_finalize": (_c_int, [_vp] * 2 + [_c_size] + [_c_int] * 6 + [_vp]),
     "fa_decode_workspace_bytes": (_c_size, [_c_int] * 5),
     "fa_decode_splitkv": (_c_int, [_vp] * 6 + [_vp, _c_size] + [_c_int] * 5 + [_c_float, _c_int, _vp]),
     "fa_check": (_c_int, [_vp]),

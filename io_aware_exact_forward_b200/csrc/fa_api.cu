@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <initializer_list>
 #include <mutex>
 
 #include "fa_status.h"
@@ -193,12 +194,115 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
   return launch_status();
 }
 
+static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
 size_t fa_backward_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int d) {
   (void)Hkv; (void)Tk;
   if (B < 0 || Hq < 1 || Tq < 0 || (d != 64 && d != 128)) return 0;
-  const size_t dq = ((size_t)B * Tq * Hq * d * 4 + 255) / 256 * 256;
-  const size_t dd = ((size_t)B * Hq * Tq * 4 + 255) / 256 * 256;
-  return dq + dd;
+  return round256((size_t)B * Tq * Hq * d * 4) + 2 * round256((size_t)B * Hq * Tq * 4);
+}
+
+// Workspace pieces of the backward pass.
+struct BwdWs {
+  float* dq_acc;
+  float* Dv;
+  float* lse2;
+};
+static BwdWs bwd_ws(void* ws, int B, int Hq, int Tq, int d) {
+  BwdWs w;
+  w.dq_acc = reinterpret_cast<float*>(ws);
+  w.Dv = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + round256((size_t)B * Tq * Hq * d * 4));
+  w.lse2 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(w.Dv) + round256((size_t)B * Hq * Tq * 4));
+  return w;
+}
+
+static int check_ws(void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d) {
+  const size_t need = fa_backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return FA_ERR_WORKSPACE;
+  return FA_OK;
+}
+
+static int check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* ptr : ptrs) {
+    if (!ptr) return FA_ERR_INVALID_ARG;
+    if (!aligned16(ptr)) return FA_ERR_ALIGNMENT;
+  }
+  return FA_OK;
+}
+
+int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void* ws, size_t ws_bytes,
+                           int B, int Hq, int Hkv, int Tq, int Tk, int d, void* stream) {
+  int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, 1.f, 0);
+  if (st) return st;
+  if (B == 0 || Tq == 0) return FA_OK;
+  if ((st = check_ptrs({o, lse, dO}))) return st;
+  if ((st = check_ws(ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d))) return st;
+  if ((st = device_setup())) return st;
+  const BwdWs w = bwd_ws(ws, B, Hq, Tq, d);
+  const long long threads = (long long)B * Tq * Hq * (d / 8);
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* o16 = reinterpret_cast<const __nv_bfloat16*>(o);
+  const __nv_bfloat16* do16 = reinterpret_cast<const __nv_bfloat16*>(dO);
+  if (d == 64)
+    fa_bwd_preprocess_kernel<64><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, w.dq_acc, B, Hq, Tq);
+  else
+    fa_bwd_preprocess_kernel<128><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, w.dq_acc, B, Hq, Tq);
+  return launch_status();
+}
+
+int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                     void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+                     float scale, int causal, void* stream) {
+  int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
+  if (st) return st;
+  if (B == 0 || Tk == 0) return FA_OK;
+  if ((st = check_ptrs({k, v, dk, dv}))) return st;
+  if (Tq > 0 && (st = check_ptrs({q, dO}))) return st;
+  if ((st = check_ws(ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d))) return st;
+  if ((st = device_setup())) return st;
+  const BwdWs w = bwd_ws(ws, B, Hq, Tq, d);
+  BwdParams p;
+  memset(&p, 0, sizeof(p));
+  if (Tq > 0) {
+    st = make_tmap_4d(&p.tm_q, q, d, Hq, Tq, B, 64, 128, true);
+    if (!st) st = make_tmap_4d(&p.tm_do, dO, d, Hq, Tq, B, 64, 128, true);
+  }
+  if (!st) st = make_tmap_4d(&p.tm_k, k, d, Hkv, Tk, B, 64, 128, true);
+  if (!st) st = make_tmap_4d(&p.tm_v, v, d, Hkv, Tk, B, 64, 128, true);
+  if (st) return st;
+  p.lse2 = w.lse2;
+  p.Dv = w.Dv;
+  p.dq_acc = w.dq_acc;
+  p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tq = Tq; p.Tk = Tk; p.causal = causal;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_kv_tiles = (Tk + 127) / 128;
+  p.wait_limit_ns = kWaitLimitNs;
+  dim3 grid(B * Hkv, p.n_kv_tiles);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    fa_bwd_dkdv_kernel<64><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+  else
+    fa_bwd_dkdv_kernel<128><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+  return launch_status();
+}
+
+int fa_backward_dq_finalize(void* dq, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk,
+                            int d, void* stream) {
+  int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, 1.f, 0);
+  if (st) return st;
+  if (B == 0 || Tq == 0) return FA_OK;
+  if ((st = check_ptrs({dq}))) return st;
+  if ((st = check_ws(ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d))) return st;
+  if ((st = device_setup())) return st;
+  const BwdWs w = bwd_ws(ws, B, Hq, Tq, d);
+  const long long n8 = (long long)B * Tq * Hq * d / 8;
+  fa_bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      w.dq_acc, reinterpret_cast<__nv_bfloat16*>(dq), n8);
+  return launch_status();
 }
 
 int fa_backward(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -207,15 +311,13 @@ int fa_backward(const void* q, const void* k, const void* v, const void* o, cons
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
   if (B == 0 || (Tq == 0 && Tk == 0)) return FA_OK;
-  if ((Tq > 0 && (!q || !o || !lse || !dO || !dq)) || (Tk > 0 && (!k || !v || !dk || !dv)))
-    return FA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
-  for (const void* ptr : ptrs)
-    if (ptr && !aligned16(ptr)) return FA_ERR_ALIGNMENT;
-  const size_t need = fa_backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d);
-  if (!ws || ws_bytes < need || !aligned16(ws)) return FA_ERR_WORKSPACE;
-  (void)stream;
-  return FA_ERR_UNSUPPORTED;
+  if (Tq > 0 && (st = check_ptrs({q, o, lse, dO, dq}))) return st;
+  if (Tk > 0 && (st = check_ptrs({k, v, dk, dv}))) return st;
+  if ((st = check_ws(ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d))) return st;
+  if ((st = fa_backward_preprocess(o, lse, dO, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream))) return st;
+  if ((st = fa_backward_dkdv(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, stream)))
+    return st;
+  return fa_backward_dq_finalize(dq, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream);
 }
 
 static size_t decode_nchunk(int Tk_max, int chunk) { return ((size_t)Tk_max + chunk - 1) / chunk; }
@@ -223,9 +325,7 @@ static size_t decode_nchunk(int Tk_max, int chunk) { return ((size_t)Tk_max + ch
 size_t fa_decode_workspace_bytes(int B, int Hq, int Tk_max, int d, int chunk) {
   if (B < 0 || Hq < 1 || Tk_max < 0 || chunk < 1 || (d != 64 && d != 128)) return 0;
   const size_t n = decode_nchunk(Tk_max, chunk);
-  const size_t wo = ((size_t)B * Hq * n * d * 4 + 255) / 256 * 256;
-  const size_t wl = ((size_t)B * Hq * n * 4 + 255) / 256 * 256;
-  return wo + wl;
+  return round256((size_t)B * Hq * n * d * 4) + round256((size_t)B * Hq * n * 4);
 }
 
 int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,

@@ -1,6 +1,483 @@
-// fa_bwd.cuh -- backward kernels (placeholder until the tcgen05 kernels land).
+// fa_bwd.cuh -- backward kernels: dQ, dK, dV of L = sum(dO * O), with S and
+// P recomputed tile by tile from the forward's log-sum-exp instead of being
+// stored ("FlashAttention" interview track, follow-up on recomputation; the
+// products dV = P^T dO, dP = dO V^T, dS = P*(dP - D), dQ = scale dS K,
+// dK = scale dS^T Q of "Efficient attention: memory-bound", section "Real
+// code moves even more").
+//
+// Three kernels:
+//   preprocess   D_i = sum_c dO_ic O_ic (fp32), LSE in log2 units (+inf for a
+//                row that saw no key, so that its P is exactly 0), dQ
+//                accumulator zeroed.                          (memory-bound)
+//   dkdv         one CTA per (128-key tile, KV head, batch).  K and V stay in
+//                shared memory; the CTA walks the query tiles of every query
+//                head of its GQA group.  Per tile, in tensor memory:
+//                  S^T = K Q^T, dP^T = V dO^T          (SS MMAs)
+//                  P^T = 2^{S^T*scale*log2e - LSE2}   (compute warps, bf16
+//                        written over S^T)
+//                  dV += P^T dO                         (TS MMA)
+//                  dS^T = P^T * (dP^T - D)             (compute warps, bf16
+//                        over dP^T and into shared memory as the A operand)
+//                  dK += dS^T Q                         (TS MMA)
+//                  dQ_tile = dS K                       (SS MMA)
+//                dQ_tile is read by a second warpgroup and added into an fp32
+//                accumulator in global memory with vector reductions (every
+//                KV tile contributes to every query row it sees).  dK and dV
+//                are summed over the group's heads in tensor memory, so the
+//                GQA sum needs no atomics.
+//   dq_convert   dq = bf16(accumulator).
+// Warp roles in dkdv: 0-3 compute (one key row per thread = TMEM lane),
+// 4-7 dQ reduction (one query row per thread), 8 MMA issuer, 9 TMA producer.
 #pragma once
+
 #include "fa_ptx.cuh"
+
 namespace fa {
-static int bwd_setup() { return FA_OK; }
+
+// ---------------------------------------------------------------------------
+// preprocess
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+    const float* __restrict__ lse, float* __restrict__ Dv, float* __restrict__ lse2,
+    float* __restrict__ dq_acc, int B, int Hq, int Tq) {
+  constexpr int LPR = D / 8;  // lanes per row, 8 elements (16 bytes) each
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = gid / LPR;            // row index in [B][Tq][Hq] order
+  const int sub = (int)(gid % LPR);
+  const long long nrows = (long long)B * Tq * Hq;
+  float dot = 0.f;
+  if (row < nrows) {
+    const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + sub * 8);
+    const uint4 c = *reinterpret_cast<const uint4*>(dO + row * D + sub * 8);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(a2[e]);
+      const float2 y = __bfloat1622float2(c2[e]);
+      dot = fmaf(x.x, y.x, dot);
+      dot = fmaf(x.y, y.y, dot);
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + sub * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+  if (row < nrows && sub == 0) {
+    const int h = (int)(row % Hq);
+    const long long bt = row / Hq;
+    const int t = (int)(bt % Tq);
+    const int b = (int)(bt / Tq);
+    const long long idx = ((long long)b * Hq + h) * Tq + t;
+    Dv[idx] = dot;
+    const float l = lse[idx];
+    lse2[idx] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dq convert
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ acc,
+                                                                __nv_bfloat16* __restrict__ dq,
+                                                                long long n8) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  uint4 out;
+  out.x = pack_bf16x2(a.x, a.y);
+  out.y = pack_bf16x2(a.z, a.w);
+  out.z = pack_bf16x2(b.x, b.y);
+  out.w = pack_bf16x2(b.z, b.w);
+  reinterpret_cast<uint4*>(dq)[i] = out;
+}
+
+// ---------------------------------------------------------------------------
+// dK / dV (+ dQ contributions)
+// ---------------------------------------------------------------------------
+struct BwdParams {
+  CUtensorMap tm_q;    // [B][Tq][Hq][d], box {64,1,128,1}, 128-byte swizzle
+  CUtensorMap tm_do;
+  CUtensorMap tm_k;    // [B][Tk][Hkv][d]
+  CUtensorMap tm_v;
+  const float* lse2;   // [B][Hq][Tq]
+  const float* Dv;     // [B][Hq][Tq]
+  float* dq_acc;       // [B][Tq][Hq][d], receives scale * dS K
+  __nv_bfloat16* dk;   // [B][Tk][Hkv][d]
+  __nv_bfloat16* dv;
+  int B, Hq, Hkv, Tq, Tk, causal;
+  float scale, scale_log2;
+  int n_kv_tiles;
+  unsigned long long wait_limit_ns;
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+template <int D>
+struct BwdCfg {
+  static constexpr int NBOX = D / 64;
+  static constexpr int BOX_BYTES = 128 * 128;
+  static constexpr int TILE = NBOX * BOX_BYTES;         // 128 rows x D bf16
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = TILE;
+  static constexpr int OFF_Q = 2 * TILE;                // 2 stages
+  static constexpr int OFF_DO = 4 * TILE;               // 2 stages
+  static constexpr int OFF_DS = 6 * TILE;               // 128 x 128 bf16, 2 boxes
+  static constexpr int OFF_LSE = OFF_DS + 2 * BOX_BYTES;  // [2][128] f32
+  static constexpr int OFF_DD = OFF_LSE + 2 * 128 * 4;    // [2][128] f32
+  static constexpr int OFF_BAR = OFF_DD + 2 * 128 * 4;
+  // kv_full, qdo_full[2], qdo_empty[2], s_full, dp_full, p_full, ds_full,
+  // dq_full, dq_free, dkdv_done, mma_done
+  static constexpr int NBAR = 13;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int THREADS = 320;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int TM_DV = 0;
+  static constexpr int TM_DK = D;
+  static constexpr int TM_S = 2 * D;
+  static constexpr int TM_DP = 2 * D + 128;
+  static constexpr int TM_DQ = (D == 128) ? TM_S : 2 * D + 256;
+  static constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);
+  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 1, 1);
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {  // the layout needs 1024-byte aligned swizzle atoms
+    if (threadIdx.x == 0) atomicCAS(&g_fa_status, 0, (int)FA_ERR_CUDA);
+    return;
+  }
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const uint32_t bar_kv = bar0;
+  auto bar_qdo_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_qdo_empty = [&](int s) { return bar0 + 8u * (3 + s); };
+  const uint32_t bar_s_full = bar0 + 8u * 5;
+  const uint32_t bar_dp_full = bar0 + 8u * 6;
+  const uint32_t bar_p_full = bar0 + 8u * 7;
+  const uint32_t bar_ds_full = bar0 + 8u * 8;
+  const uint32_t bar_dq_full = bar0 + 8u * 9;
+  const uint32_t bar_dq_free = bar0 + 8u * 10;
+  const uint32_t bar_dkdv_done = bar0 + 8u * 11;
+  const uint32_t bar_mma_done = bar0 + 8u * 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
+  float* dd_s = reinterpret_cast<float*>(smem + C::OFF_DD);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int hb = blockIdx.x;                 // (batch, kv head), fastest
+  const int b = hb / p.Hkv;
+  const int hkv = hb % p.Hkv;
+  const int kt = blockIdx.y;                 // heaviest (first) key tiles first
+  const int j0 = kt * 128;
+  const int G = p.Hq / p.Hkv;
+  const int n_qt = (p.Tq + 127) / 128;
+  int qt_begin = 0;
+  if (p.causal) {
+    const int qmin = j0 - (p.Tk - p.Tq);     // first query that sees key j0
+    qt_begin = qmin <= 0 ? 0 : min(n_qt, qmin / 128);
+  }
+  const int nq = n_qt - qt_begin;
+  const int n_it = G * nq;
+  WaitCtl wc{abort_flag, p.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_qdo_full(s), 32);
+      mbar_init(bar_qdo_empty(s), 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_p_full, 128);
+    mbar_init(bar_ds_full, 128);
+    mbar_init(bar_dq_full, 1);
+    mbar_init(bar_dq_free, 128);
+    mbar_init(bar_dkdv_done, 1);
+    mbar_init(bar_mma_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    bool ok = true;
+    int issued = 0;
+    if (n_it > 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_do);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_v);
+        mbar_arrive_expect_tx(bar_kv, 2 * C::TILE);
+        for (int kb = 0; kb < C::NBOX; ++kb) {
+          tma_load_4d(sbase + C::OFF_K + kb * C::BOX_BYTES, &p.tm_k, bar_kv, kb * 64, hkv, j0, b);
+          tma_load_4d(sbase + C::OFF_V + kb * C::BOX_BYTES, &p.tm_v, bar_kv, kb * 64, hkv, j0, b);
+        }
+      }
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it & 1;
+        const int h = hkv * G + it / nq;
+        const int q0 = (qt_begin + it % nq) * 128;
+        if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_empty(s), ((it >> 1) - 1) & 1, wc));
+        if (!ok) break;
+        // per-row statistics of this query tile (4 rows per lane)
+        const size_t rbase = ((size_t)b * p.Hq + h) * p.Tq;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = lane * 4 + e;
+          const int q = q0 + r;
+          lse_s[s * 128 + r] = q < p.Tq ? p.lse2[rbase + q] : INFINITY;
+          dd_s[s * 128 + r] = q < p.Tq ? p.Dv[rbase + q] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_qdo_full(s), 2 * C::TILE);
+          for (int kb = 0; kb < C::NBOX; ++kb) {
+            tma_load_4d(sbase + C::OFF_Q + s * C::TILE + kb * C::BOX_BYTES, &p.tm_q, bar_qdo_full(s),
+                        kb * 64, h, q0, b);
+            tma_load_4d(sbase + C::OFF_DO + s * C::TILE + kb * C::BOX_BYTES, &p.tm_do, bar_qdo_full(s),
+                        kb * 64, h, q0, b);
+          }
+        } else {
+          mbar_arrive(bar_qdo_full(s));
+        }
+        ++issued;
+      }
+      if (!ok && lane == 0) {
+        mbar_wait_drain(bar_kv, 0, p.wait_limit_ns);
+        for (int it = max(0, issued - 2); it < issued; ++it)
+          mbar_wait_drain(bar_qdo_full(it & 1), (it >> 1) & 1, p.wait_limit_ns);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_it > 0) {
+      const uint32_t tS = tmem + C::TM_S, tDP = tmem + C::TM_DP, tDV = tmem + C::TM_DV,
+                     tDK = tmem + C::TM_DK, tDQ = tmem + C::TM_DQ;
+      const uint32_t aK = sbase + C::OFF_K, aV = sbase + C::OFF_V, aDS = sbase + C::OFF_DS;
+      auto kdesc = [&](uint32_t base, int k) {  // K-major tile, k-th 16-element slice of d
+        return smem_desc_sw128(base + (k >> 2) * C::BOX_BYTES + (k & 3) * 32, 16, 1024);
+      };
+      auto mndesc = [&](uint32_t base, int k) {  // MN-major view, k-th 16-row slice
+        return smem_desc_sw128(base + k * 16 * 128, C::BOX_BYTES, 1024);
+      };
+      bool ok = mbar_wait(bar_kv, 0, wc);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it & 1;
+        const uint32_t aQ = sbase + C::OFF_Q + s * C::TILE, aDO = sbase + C::OFF_DO + s * C::TILE;
+        ok = mbar_wait(bar_qdo_full(s), (it >> 1) & 1, wc);
+        if (!ok) break;
+        if (D == 128 && it > 0) {
+          ok = mbar_wait(bar_dq_free, (it - 1) & 1, wc);
+          if (!ok) break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) mma_ss(tS, kdesc(aK, k), kdesc(aQ, k), C::IDESC_SS, k > 0);
+        mma_commit(bar_s_full);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc(aV, k), kdesc(aDO, k), C::IDESC_SS, k > 0);
+        mma_commit(bar_dp_full);
+        ok = mbar_wait(bar_p_full, it & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mma_ts(tDV, tS + k * 8, mndesc(aDO, k), C::IDESC_TS, it > 0 || k > 0);
+        ok = mbar_wait(bar_ds_full, it & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mma_ts(tDK, tDP + k * 8, mndesc(aQ, k), C::IDESC_TS, it > 0 || k > 0);
+        mma_commit(bar_qdo_empty(s));
+        if (D == 64 && it > 0) {
+          ok = mbar_wait(bar_dq_free, (it - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK, k), C::IDESC_DQ, k > 0);
+        mma_commit(bar_dq_full);
+      }
+      if (ok) mma_commit(bar_dkdv_done);
+      mma_commit(bar_mma_done);
+      mbar_wait_drain(bar_mma_done, 0, p.wait_limit_ns);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ compute
+    const int j = threadIdx.x;               // key row in the tile == TMEM lane
+    const int key = j0 + j;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t tS = tmem + C::TM_S + lane_off;
+    const uint32_t tDP = tmem + C::TM_DP + lane_off;
+    const int qmin = key - (p.Tk - p.Tq);   // causal: first query that sees this key
+    const bool key_ok = key < p.Tk;
+    uint8_t* ds_row = smem + C::OFF_DS + j * 128;
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int s = it & 1;
+      const int q0 = (qt_begin + it % nq) * 128;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), (it >> 1) & 1, wc));
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, it & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t su[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, su + c * 32);
+      tmem_wait_ld();
+      const float* lrow = lse_s + s * 128;
+      const int cmin = p.causal ? qmin - q0 : 0;  // columns < cmin are masked
+      // P^T = 2^{S*scale*log2e - LSE2}, packed to bf16 pairs in place.
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        float p0 = ex2_approx(fmaf(__uint_as_float(su[2 * c]), p.scale_log2, -lrow[2 * c]));
+        float p1 = ex2_approx(fmaf(__uint_as_float(su[2 * c + 1]), p.scale_log2, -lrow[2 * c + 1]));
+        if (!key_ok || 2 * c < cmin) p0 = 0.f;
+        if (!key_ok || 2 * c + 1 < cmin) p1 = 0.f;
+        su[c] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(tS, su);
+      tmem_st32(tS + 32, su + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p_full);
+
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, it & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      const float* drow = dd_s + s * 128;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t dp[32];
+        tmem_ld32(tDP + c4 * 32, dp);
+        tmem_wait_ld();
+        uint32_t ds[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(&su[c4 * 16 + e]);
+          const float2 pf = __bfloat1622float2(pp);
+          const int col = c4 * 32 + 2 * e;
+          const float d0 = pf.x * (__uint_as_float(dp[2 * e]) - drow[col]);
+          const float d1 = pf.y * (__uint_as_float(dp[2 * e + 1]) - drow[col + 1]);
+          ds[e] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tDP + c4 * 16, ds);
+        // dS into shared memory: row j of box (c4/2), 16-byte chunks
+        // 4*(c4%2) .. +3, 128-byte swizzle (chunk ^ (row % 8)).
+        uint8_t* box = ds_row + (c4 >> 1) * C::BOX_BYTES;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int chunk = 4 * (c4 & 1) + cc;
+          *reinterpret_cast<uint4*>(box + ((chunk ^ (j & 7)) << 4)) =
+              make_uint4(ds[4 * cc], ds[4 * cc + 1], ds[4 * cc + 2], ds[4 * cc + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_ds_full);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (n_it > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dkdv_done, 0, wc));
+    tc_fence_after();
+    const bool have = n_it > 0 && ok;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off;
+      const float mul = which ? p.scale : 1.f;
+      __nv_bfloat16* dst = (which ? p.dk : p.dv) + (((size_t)b * p.Tk + (key < p.Tk ? key : 0)) * p.Hkv + hkv) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        if (have) {
+          tmem_ld32(tsrc + c * 32, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        uint4 pk[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pw[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+        if (key < p.Tk) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ reduction
+    const int r = threadIdx.x - 128;         // query row in the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tDQ = tmem + C::TM_DQ + lane_off;
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int h = hkv * G + it / nq;
+      const int q = (qt_begin + it % nq) * 128 + r;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_dq_full, it & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      float* dst = p.dq_acc + (((size_t)b * p.Tq + (q < p.Tq ? q : 0)) * p.Hq + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tDQ + c * 32, v);
+        tmem_wait_ld();
+        if (q < p.Tq) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
+                       __uint_as_float(v[4 * e + 1]) * p.scale, __uint_as_float(v[4 * e + 2]) * p.scale,
+                       __uint_as_float(v[4 * e + 3]) * p.scale);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_dq_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+static int bwd_setup() {
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64>),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<64>::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128>),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<128>::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 }  // namespace fa

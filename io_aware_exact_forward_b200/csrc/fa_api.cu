@@ -63,6 +63,22 @@ static int make_tmap_4d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t 
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// 4-D fp32 tensor [n3][n2][n1][n0] with box {32, 1, 128, 1} and the 128-byte
+// swizzle (the dQ accumulator, written by bulk tensor reduce-add).
+static int make_tmap_f32_4d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
+                            uint64_t n3) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {n0, n1, n2, n3};
+  const cuuint64_t strides[3] = {n0 * 4, n0 * n1 * 4, n0 * n1 * n2 * 4};
+  const cuuint32_t box[4] = {32, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Per-device set-up: architecture check and shared-memory opt-in, once.
 // ---------------------------------------------------------------------------
@@ -135,8 +151,9 @@ static int check_prefill(int B, int Hq, int Hkv, int Tq, int Tk, int d, float sc
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (!isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  // Tensor-map extents are 32-bit and row indices are int.
-  if ((int64_t)Tq > (1 << 30) || (int64_t)Tk > (1 << 30) || (int64_t)B * Hq > (1 << 30))
+  // Tensor-map extents are 32-bit and row indices are int; (batch, head)
+  // pairs index the second grid dimension (at most 65535).
+  if ((int64_t)Tq > (1 << 30) || (int64_t)Tk > (1 << 30) || (int64_t)B * Hq > 65535)
     return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
@@ -185,7 +202,7 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_mblocks = (Tq + 255) / 256;
   p.wait_limit_ns = kWaitLimitNs;
-  dim3 grid(B * Hq, p.n_mblocks);
+  dim3 grid(p.n_mblocks, B * Hq);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64)
     fa_fwd_kernel<64><<<grid, FwdCfg<64>::THREADS, FwdCfg<64>::SMEM_BYTES, s>>>(p);
@@ -270,6 +287,7 @@ int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO
   }
   if (!st) st = make_tmap_4d(&p.tm_k, k, d, Hkv, Tk, B, 64, 128, true);
   if (!st) st = make_tmap_4d(&p.tm_v, v, d, Hkv, Tk, B, 64, 128, true);
+  if (!st && Tq > 0) st = make_tmap_f32_4d(&p.tm_dq, w.dq_acc, d, Hq, Tq, B);
   if (st) return st;
   p.lse2 = w.lse2;
   p.Dv = w.Dv;
@@ -281,7 +299,7 @@ int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_kv_tiles = (Tk + 127) / 128;
   p.wait_limit_ns = kWaitLimitNs;
-  dim3 grid(B * Hkv, p.n_kv_tiles);
+  dim3 grid(p.n_kv_tiles, B * Hkv);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64)
     fa_bwd_dkdv_kernel<64><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);

@@ -100,10 +100,11 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __r
 // dK / dV (+ dQ contributions)
 // ---------------------------------------------------------------------------
 struct BwdParams {
-  CUtensorMap tm_q;    // [B][Tq][Hq][d], box {64,1,128,1}, 128-byte swizzle
+  CUtensorMap tm_q;    // [B][Tq][Hq][d] bf16, box {64,1,128,1}, 128-byte swizzle
   CUtensorMap tm_do;
   CUtensorMap tm_k;    // [B][Tk][Hkv][d]
   CUtensorMap tm_v;
+  CUtensorMap tm_dq;   // fp32 accumulator [B][Tq][Hq][d], box {32,1,128,1}, 128-byte swizzle
   const float* lse2;   // [B][Hq][Tq]
   const float* Dv;     // [B][Hq][Tq]
   float* dq_acc;       // [B][Tq][Hq][d], receives scale * dS K
@@ -121,38 +122,60 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+// Bulk tensor reduce-add of a shared-memory tile into global memory (fp32).
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* m, uint32_t src, int c0, int c1,
+                                                  int c2, int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 template <int D>
 struct BwdCfg {
   static constexpr int NBOX = D / 64;
   static constexpr int BOX_BYTES = 128 * 128;
   static constexpr int TILE = NBOX * BOX_BYTES;         // 128 rows x D bf16
+  // d = 64: two S^T buffers in tensor memory and dQ leaves through a shared-
+  // memory tile and a bulk tensor reduce.  d = 128: one S^T buffer (tensor
+  // memory is full) and dQ leaves through vector reductions.
+  static constexpr int NSBUF = (D == 64) ? 2 : 1;
+  static constexpr bool DQ_TMA = (D == 64);
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = TILE;
   static constexpr int OFF_Q = 2 * TILE;                // 2 stages
   static constexpr int OFF_DO = 4 * TILE;               // 2 stages
   static constexpr int OFF_DS = 6 * TILE;               // 128 x 128 bf16, 2 boxes
-  static constexpr int OFF_LSE = OFF_DS + 2 * BOX_BYTES;  // [2][128] f32
-  static constexpr int OFF_DD = OFF_LSE + 2 * 128 * 4;    // [2][128] f32
+  static constexpr int OFF_DQS = OFF_DS + 2 * BOX_BYTES;  // fp32 128 x D staging (DQ_TMA only)
+  static constexpr int DQS_BYTES = DQ_TMA ? 128 * D * 4 : 0;
+  static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;   // [2][128] f32
+  static constexpr int OFF_DD = OFF_LSE + 2 * 128 * 4;  // [2][128] f32
   static constexpr int OFF_BAR = OFF_DD + 2 * 128 * 4;
-  // kv_full, qdo_full[2], qdo_empty[2], s_full, dp_full, p_full, ds_full,
-  // dq_full, dq_free, dkdv_done, mma_done
-  static constexpr int NBAR = 13;
+  // kv_full, qdo_full[2], qdo_empty[2], s_full[2], p_full[2], dp_full, ds_full,
+  // dq_full[2], dq_free[2], dkdv_done, mma_done
+  static constexpr int NBAR = 17;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 448;                   // 3 warpgroups + MMA warp + TMA warp
   static constexpr int TMEM_COLS = 512;
   static constexpr int TM_DV = 0;
   static constexpr int TM_DK = D;
-  static constexpr int TM_S = 2 * D;
-  static constexpr int TM_DP = 2 * D + 128;
-  static constexpr int TM_DQ = (D == 128) ? TM_S : 2 * D + 256;
+  static constexpr int TM_S0 = 2 * D;                   // S^T buffers; dQ reuses them
+  static constexpr int TM_DP = 2 * D + 128 * NSBUF;
   static constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 1, 1);
+  static_assert(TM_DP + 128 <= TMEM_COLS, "tensor memory overflow");
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -164,14 +187,14 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_consta
   const uint32_t bar_kv = bar0;
   auto bar_qdo_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto bar_qdo_empty = [&](int s) { return bar0 + 8u * (3 + s); };
-  const uint32_t bar_s_full = bar0 + 8u * 5;
-  const uint32_t bar_dp_full = bar0 + 8u * 6;
-  const uint32_t bar_p_full = bar0 + 8u * 7;
-  const uint32_t bar_ds_full = bar0 + 8u * 8;
-  const uint32_t bar_dq_full = bar0 + 8u * 9;
-  const uint32_t bar_dq_free = bar0 + 8u * 10;
-  const uint32_t bar_dkdv_done = bar0 + 8u * 11;
-  const uint32_t bar_mma_done = bar0 + 8u * 12;
+  auto bar_s_full = [&](int b) { return bar0 + 8u * (5 + b); };
+  auto bar_p_full = [&](int b) { return bar0 + 8u * (7 + b); };
+  const uint32_t bar_dp_full = bar0 + 8u * 9;
+  const uint32_t bar_ds_full = bar0 + 8u * 10;
+  auto bar_dq_full = [&](int b) { return bar0 + 8u * (11 + b); };
+  auto bar_dq_free = [&](int b) { return bar0 + 8u * (13 + b); };
+  const uint32_t bar_dkdv_done = bar0 + 8u * 15;
+  const uint32_t bar_mma_done = bar0 + 8u * 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -179,10 +202,12 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_consta
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int hb = blockIdx.x;                 // (batch, kv head), fastest
+  // Key tiles of one (batch, KV head) are adjacent in launch order, so the
+  // head's dQ accumulator rows and Q/dO tiles stay in L2 while they run.
+  const int kt = blockIdx.x;
+  const int hb = blockIdx.y;
   const int b = hb / p.Hkv;
   const int hkv = hb % p.Hkv;
-  const int kt = blockIdx.y;                 // heaviest (first) key tiles first
   const int j0 = kt * 128;
   const int G = p.Hq / p.Hkv;
   const int n_qt = (p.Tq + 127) / 128;
@@ -201,18 +226,18 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_consta
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_qdo_full(s), 32);
       mbar_init(bar_qdo_empty(s), 1);
+      mbar_init(bar_s_full(s), 1);
+      mbar_init(bar_p_full(s), 128);
+      mbar_init(bar_dq_full(s), 1);
+      mbar_init(bar_dq_free(s), 128);
     }
-    mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
-    mbar_init(bar_p_full, 128);
     mbar_init(bar_ds_full, 128);
-    mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_free, 128);
     mbar_init(bar_dkdv_done, 1);
     mbar_init(bar_mma_done, 1);
     fence_barrier_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -220,8 +245,10 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  auto it_head = [&](int it) { return hkv * G + it / nq; };
+  auto it_q0 = [&](int it) { return (qt_begin + it % nq) * 128; };
 
-  if (warp == 9) {
+  if (warp == 13) {
     // ------------------------------------------------------------ producer
     bool ok = true;
     int issued = 0;
@@ -239,11 +266,10 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_consta
       }
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it & 1;
-        const int h = hkv * G + it / nq;
-        const int q0 = (qt_begin + it % nq) * 128;
+        const int h = it_head(it);
+        const int q0 = it_q0(it);
         if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_empty(s), ((it >> 1) - 1) & 1, wc));
         if (!ok) break;
-        // per-row statistics of this query tile (4 rows per lane)
         const size_t rbase = ((size_t)b * p.Hq + h) * p.Tq;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -272,135 +298,128 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_consta
           mbar_wait_drain(bar_qdo_full(it & 1), (it >> 1) & 1, p.wait_limit_ns);
       }
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_it > 0) {
-      const uint32_t tS = tmem + C::TM_S, tDP = tmem + C::TM_DP, tDV = tmem + C::TM_DV,
-                     tDK = tmem + C::TM_DK, tDQ = tmem + C::TM_DQ;
+      const uint32_t tDP = tmem + C::TM_DP, tDV = tmem + C::TM_DV, tDK = tmem + C::TM_DK;
+      auto tS = [&](int buf) { return tmem + C::TM_S0 + 128 * buf; };
       const uint32_t aK = sbase + C::OFF_K, aV = sbase + C::OFF_V, aDS = sbase + C::OFF_DS;
+      auto aQ = [&](int it) { return sbase + C::OFF_Q + (it & 1) * C::TILE; };
+      auto aDO = [&](int it) { return sbase + C::OFF_DO + (it & 1) * C::TILE; };
       auto kdesc = [&](uint32_t base, int k) {  // K-major tile, k-th 16-element slice of d
         return smem_desc_sw128(base + (k >> 2) * C::BOX_BYTES + (k & 3) * 32, 16, 1024);
       };
       auto mndesc = [&](uint32_t base, int k) {  // MN-major view, k-th 16-row slice
         return smem_desc_sw128(base + k * 16 * 128, C::BOX_BYTES, 1024);
       };
-      bool ok = mbar_wait(bar_kv, 0, wc);
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int s = it & 1;
-        const uint32_t aQ = sbase + C::OFF_Q + s * C::TILE, aDO = sbase + C::OFF_DO + s * C::TILE;
-        ok = mbar_wait(bar_qdo_full(s), (it >> 1) & 1, wc);
-        if (!ok) break;
-        if (D == 128 && it > 0) {
-          ok = mbar_wait(bar_dq_free, (it - 1) & 1, wc);
-          if (!ok) break;
-        }
-        tc_fence_after();
+      auto issue_s = [&](int it) {
+        const int buf = it % C::NSBUF;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss(tS, kdesc(aK, k), kdesc(aQ, k), C::IDESC_SS, k > 0);
-        mma_commit(bar_s_full);
+        for (int k = 0; k < D / 16; ++k) mma_ss(tS(buf), kdesc(aK, k), kdesc(aQ(it), k), C::IDESC_SS, k > 0);
+        mma_commit(bar_s_full(buf));
+      };
+      auto issue_dp = [&](int it) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc(aV, k), kdesc(aDO, k), C::IDESC_SS, k > 0);
+        for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc(aV, k), kdesc(aDO(it), k), C::IDESC_SS, k > 0);
         mma_commit(bar_dp_full);
-        ok = mbar_wait(bar_p_full, it & 1, wc);
+      };
+      bool ok = mbar_wait(bar_kv, 0, wc);
+      if (ok) ok = mbar_wait(bar_qdo_full(0), 0, wc);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int buf = it % C::NSBUF;
+        if (C::NSBUF == 2 && it + 1 < n_it) {
+          // S^T of the next tile into the other buffer, which dQ(it-1) used.
+          ok = mbar_wait(bar_qdo_full((it + 1) & 1), ((it + 1) >> 1) & 1, wc);
+          if (ok && it >= 1) ok = mbar_wait(bar_dq_free((it + 1) & 1), ((it - 1) >> 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(it + 1);
+        }
+        ok = mbar_wait(bar_p_full(buf), (it / C::NSBUF) & 1, wc);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mma_ts(tDV, tS + k * 8, mndesc(aDO, k), C::IDESC_TS, it > 0 || k > 0);
+        for (int k = 0; k < 8; ++k)
+          mma_ts(tDV, tS(buf) + k * 8, mndesc(aDO(it), k), C::IDESC_TS, it > 0 || k > 0);
         ok = mbar_wait(bar_ds_full, it & 1, wc);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mma_ts(tDK, tDP + k * 8, mndesc(aQ, k), C::IDESC_TS, it > 0 || k > 0);
-        mma_commit(bar_qdo_empty(s));
-        if (D == 64 && it > 0) {
-          ok = mbar_wait(bar_dq_free, (it - 1) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-        }
+        for (int k = 0; k < 8; ++k)
+          mma_ts(tDK, tDP + k * 8, mndesc(aQ(it), k), C::IDESC_TS, it > 0 || k > 0);
+        mma_commit(bar_qdo_empty(it & 1));
+        // dQ(it) = dS K into the S^T buffer of this tile (P^T consumed above).
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK, k), C::IDESC_DQ, k > 0);
-        mma_commit(bar_dq_full);
+        for (int k = 0; k < 8; ++k) mma_ss(tS(buf), mndesc(aDS, k), mndesc(aK, k), C::IDESC_DQ, k > 0);
+        mma_commit(bar_dq_full(buf));
+        if (it + 1 < n_it) {
+          if (C::NSBUF == 1) {
+            ok = mbar_wait(bar_qdo_full((it + 1) & 1), ((it + 1) >> 1) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_dp(it + 1);
+          if (C::NSBUF == 1) {
+            ok = mbar_wait(bar_dq_free(0), it & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(it + 1);
+          }
+        }
       }
       if (ok) mma_commit(bar_dkdv_done);
       mma_commit(bar_mma_done);
       mbar_wait_drain(bar_mma_done, 0, p.wait_limit_ns);
     }
   } else if (warp < 4) {
-    // ------------------------------------------------------------ compute
+    // ------------------------------------------------------------ P^T (WG-A)
     const int j = threadIdx.x;               // key row in the tile == TMEM lane
     const int key = j0 + j;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t tS = tmem + C::TM_S + lane_off;
-    const uint32_t tDP = tmem + C::TM_DP + lane_off;
-    const int qmin = key - (p.Tk - p.Tq);   // causal: first query that sees this key
+    const int qmin = key - (p.Tk - p.Tq);    // causal: first query that sees this key
     const bool key_ok = key < p.Tk;
-    uint8_t* ds_row = smem + C::OFF_DS + j * 128;
+    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
-      const int s = it & 1;
-      const int q0 = (qt_begin + it % nq) * 128;
+      const int s = it & 1, buf = it % C::NSBUF;
+      const int q0 = it_q0(it);
+      const uint32_t tS = tmem + C::TM_S0 + 128 * buf + lane_off;
       ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), (it >> 1) & 1, wc));
-      if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, it & 1, wc));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(buf), (it / C::NSBUF) & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      uint32_t su[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, su + c * 32);
-      tmem_wait_ld();
       const float* lrow = lse_s + s * 128;
       const int cmin = p.causal ? qmin - q0 : 0;  // columns < cmin are masked
-      // P^T = 2^{S*scale*log2e - LSE2}, packed to bf16 pairs in place.
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float p0 = ex2_approx(fmaf(__uint_as_float(su[2 * c]), p.scale_log2, -lrow[2 * c]));
-        float p1 = ex2_approx(fmaf(__uint_as_float(su[2 * c + 1]), p.scale_log2, -lrow[2 * c + 1]));
-        if (!key_ok || 2 * c < cmin) p0 = 0.f;
-        if (!key_ok || 2 * c + 1 < cmin) p1 = 0.f;
-        su[c] = pack_bf16x2(p0, p1);
-      }
-      tmem_st32(tS, su);
-      tmem_st32(tS + 32, su + 32);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p_full);
-
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, it & 1, wc));
-      if (!ok) break;
-      tc_fence_after();
-      const float* drow = dd_s + s * 128;
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t dp[32];
-        tmem_ld32(tDP + c4 * 32, dp);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(tS + c * 32, sv);
         tmem_wait_ld();
-        uint32_t ds[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(&su[c4 * 16 + e]);
-          const float2 pf = __bfloat1622float2(pp);
-          const int col = c4 * 32 + 2 * e;
-          const float d0 = pf.x * (__uint_as_float(dp[2 * e]) - drow[col]);
-          const float d1 = pf.y * (__uint_as_float(dp[2 * e + 1]) - drow[col + 1]);
-          ds[e] = pack_bf16x2(d0, d1);
+          const int col = c * 32 + 2 * e;
+          const float2 l2 = *reinterpret_cast<const float2*>(lrow + col);
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                                      sl2, make_float2(-l2.x, -l2.y));
+          float p0 = ex2_approx(x.x);
+          float p1 = ex2_approx(x.y);
+          if (!key_ok || col < cmin) p0 = 0.f;
+          if (!key_ok || col + 1 < cmin) p1 = 0.f;
+          pk[e] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tDP + c4 * 16, ds);
-        // dS into shared memory: row j of box (c4/2), 16-byte chunks
-        // 4*(c4%2) .. +3, 128-byte swizzle (chunk ^ (row % 8)).
-        uint8_t* box = ds_row + (c4 >> 1) * C::BOX_BYTES;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int chunk = 4 * (c4 & 1) + cc;
-          *reinterpret_cast<uint4*>(box + ((chunk ^ (j & 7)) << 4)) =
-              make_uint4(ds[4 * cc], ds[4 * cc + 1], ds[4 * cc + 2], ds[4 * cc + 3]);
-        }
+        tmem_st16(tS + c * 16, pk);
       }
       tmem_wait_st();
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar_ds_full);
+      mbar_arrive(bar_p_full(buf));
     }
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ dK, dV out
     if (n_it > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dkdv_done, 0, wc));
     tc_fence_after();
     const bool have = n_it > 0 && ok;
@@ -431,40 +450,121 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dkdv_kernel(const __grid_consta
         }
       }
     }
-  } else {
-    // ------------------------------------------------------------ dQ reduction
-    const int r = threadIdx.x - 128;         // query row in the tile == TMEM lane
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ dS (WG-B)
+    const int j = threadIdx.x - 128;         // key row == TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tDQ = tmem + C::TM_DQ + lane_off;
+    const uint32_t tDP = tmem + C::TM_DP + lane_off;
+    uint8_t* ds_row = smem + C::OFF_DS + j * 128;
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
-      const int h = hkv * G + it / nq;
-      const int q = (qt_begin + it % nq) * 128 + r;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_dq_full, it & 1, wc));
+      const int s = it & 1, buf = it % C::NSBUF;
+      const uint32_t tP = tmem + C::TM_S0 + 128 * buf + lane_off;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), (it >> 1) & 1, wc));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_p_full(buf), (it / C::NSBUF) & 1, wc));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, it & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      float* dst = p.dq_acc + (((size_t)b * p.Tq + (q < p.Tq ? q : 0)) * p.Hq + h) * D;
+      const float* drow = dd_s + s * 128;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tDQ + c * 32, v);
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t pp[16], dp[32];
+        tmem_ld16(tP + c4 * 16, pp);
+        tmem_ld32(tDP + c4 * 32, dp);
         tmem_wait_ld();
-        if (q < p.Tq) {
+        uint32_t ds[16];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
-                       __uint_as_float(v[4 * e + 1]) * p.scale, __uint_as_float(v[4 * e + 2]) * p.scale,
-                       __uint_as_float(v[4 * e + 3]) * p.scale);
+        for (int e = 0; e < 16; ++e) {
+          const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[e]));
+          const float2 dd = *reinterpret_cast<const float2*>(drow + c4 * 32 + 2 * e);
+          const float2 t = __fadd2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                                      make_float2(-dd.x, -dd.y));
+          const float2 r = __fmul2_rn(pf, t);
+          ds[e] = pack_bf16x2(r.x, r.y);
+        }
+        tmem_st16(tDP + c4 * 16, ds);
+        // dS into shared memory: row j of box (c4/2), 16-byte chunks
+        // 4*(c4%2) .. +3, 128-byte swizzle (chunk ^ (row % 8)).
+        uint8_t* box = ds_row + (c4 >> 1) * C::BOX_BYTES;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int chunk = 4 * (c4 & 1) + cc;
+          *reinterpret_cast<uint4*>(box + ((chunk ^ (j & 7)) << 4)) =
+              make_uint4(ds[4 * cc], ds[4 * cc + 1], ds[4 * cc + 2], ds[4 * cc + 3]);
         }
       }
+      tmem_wait_st();
+      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar_dq_free);
+      mbar_arrive(bar_ds_full);
+    }
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ dQ (WG-C)
+    const int r = threadIdx.x - 256;         // query row in the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int buf = it % C::NSBUF;
+      const int h = it_head(it);
+      const int q0 = it_q0(it);
+      const uint32_t tDQ = tmem + C::TM_S0 + 128 * buf + lane_off;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_dq_full(buf), (it / C::NSBUF) & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      if constexpr (C::DQ_TMA) {
+        uint32_t v[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tDQ + c * 32, v + c * 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_dq_free(buf));
+        // The previous tile's bulk reduce must have read the staging tile.
+        if (threadIdx.x == 256) bulk_wait_group_read0();
+        named_bar_sync(2, 128);
+        // fp32 staging, boxes of 32 columns, 128-byte swizzle.
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) {
+          const int box = c >> 3, chunk = c & 7;
+          *reinterpret_cast<float4*>(smem + C::OFF_DQS + box * (128 * 128) + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+              make_float4(__uint_as_float(v[4 * c]) * p.scale, __uint_as_float(v[4 * c + 1]) * p.scale,
+                          __uint_as_float(v[4 * c + 2]) * p.scale, __uint_as_float(v[4 * c + 3]) * p.scale);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(2, 128);
+        if (threadIdx.x == 256) {
+#pragma unroll
+          for (int box = 0; box < D / 32; ++box)
+            tma_reduce_add_4d(&p.tm_dq, sbase + C::OFF_DQS + box * (128 * 128), box * 32, h, q0, b);
+          bulk_commit_group();
+        }
+      } else {
+        const int q = q0 + r;
+        float* dst = p.dq_acc + (((size_t)b * p.Tq + (q < p.Tq ? q : 0)) * p.Hq + h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tDQ + c * 32, v);
+          tmem_wait_ld();
+          if (q < p.Tq) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
+                         __uint_as_float(v[4 * e + 1]) * p.scale, __uint_as_float(v[4 * e + 2]) * p.scale,
+                         __uint_as_float(v[4 * e + 3]) * p.scale);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_dq_free(buf));
+      }
+    }
+    if constexpr (C::DQ_TMA) {
+      if (threadIdx.x == 256) bulk_wait_group0();
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

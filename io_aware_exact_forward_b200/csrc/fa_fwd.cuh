@@ -87,12 +87,14 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
+  // Query blocks of one (batch, head) are adjacent in launch order, so they
+  // share that head's K/V tiles through L2; within a head the heaviest
+  // causal block (the last one) goes first.
+  const int bh = blockIdx.y;
   const int b = bh / p.Hq;
   const int h = bh % p.Hq;
   const int hkv = h / (p.Hq / p.Hkv);
-  // Heaviest causal blocks first: blockIdx.y = 0 is the last query block.
-  const int mblock = p.n_mblocks - 1 - (int)blockIdx.y;
+  const int mblock = p.n_mblocks - 1 - (int)blockIdx.x;
   const int m0 = mblock * 2 * C::BM;
 
   // Number of KV tiles this CTA visits.

@@ -86,9 +86,9 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
 
 /*
  * Bytes of device workspace fa_backward needs: an fp32 dQ accumulator
- * [B,Tq,Hq,d], the fp32 row terms D_i = sum_c dO_ic O_ic [B,Hq,Tq] and the
- * LSE in log2 units [B,Hq,Tq], each rounded up to 256 bytes.  Returns 0 for
- * invalid sizes.
+ * [B,Tq,Hq,d], the fp32 row terms D_i = sum_c dO_ic O_ic and the LSE in log2
+ * units, each [B,Hq,Tq_pad] with Tq_pad = Tq rounded up to 128; every piece
+ * rounded up to 256 bytes.  Returns 0 for invalid sizes.
  */
 size_t fa_backward_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int d);
 

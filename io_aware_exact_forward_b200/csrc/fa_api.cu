@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <initializer_list>
 #include <mutex>
 
@@ -138,6 +139,20 @@ static int device_setup() {
   return state[dev] - 1;
 }
 
+// Number of SMs of the current device (persistent grids use one CTA per SM).
+static int sm_count(int* n) {
+  static int cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return FA_ERR_CUDA;
+    cache[dev] = v;
+  }
+  *n = cache[dev];
+  return FA_OK;
+}
+
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static int launch_status() {
@@ -151,9 +166,10 @@ static int check_prefill(int B, int Hq, int Hkv, int Tq, int Tk, int d, float sc
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (!isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  // Tensor-map extents are 32-bit and row indices are int; (batch, head)
-  // pairs index the second grid dimension (at most 65535).
-  if ((int64_t)Tq > (1 << 30) || (int64_t)Tk > (1 << 30) || (int64_t)B * Hq > 65535)
+  // Tensor-map extents are 32-bit and row/item indices are int; (batch, KV
+  // head) pairs index the backward's second grid dimension (at most 65535).
+  if ((int64_t)Tq > (1 << 30) || (int64_t)Tk > (1 << 30) || (int64_t)B * Hq > 65535 ||
+      (int64_t)B * Hq * ((Tq + 255) / 256) > (1ll << 30))
     return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
@@ -201,8 +217,14 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_mblocks = (Tq + 255) / 256;
+  p.n_items = B * Hq * p.n_mblocks;
   p.wait_limit_ns = kWaitLimitNs;
-  dim3 grid(p.n_mblocks, B * Hq);
+  // Uniform (non-causal) items: persistent, one CTA per SM.  Causal items
+  // differ in cost: one CTA per item, heaviest first, balanced by the block
+  // scheduler.
+  int nsm = 0;
+  if ((st = sm_count(&nsm))) return st;
+  dim3 grid(causal ? p.n_items : std::min(p.n_items, nsm));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64)
     fa_fwd_kernel<64><<<grid, FwdCfg<64>::THREADS, FwdCfg<64>::SMEM_BYTES, s>>>(p);
@@ -213,10 +235,12 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
 
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
+static int tq_pad(int Tq) { return (Tq + 127) / 128 * 128; }
+
 size_t fa_backward_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int d) {
   (void)Hkv; (void)Tk;
   if (B < 0 || Hq < 1 || Tq < 0 || (d != 64 && d != 128)) return 0;
-  return round256((size_t)B * Tq * Hq * d * 4) + 2 * round256((size_t)B * Hq * Tq * 4);
+  return round256((size_t)B * Tq * Hq * d * 4) + 2 * round256((size_t)B * Hq * tq_pad(Tq) * 4);
 }
 
 // Workspace pieces of the backward pass.
@@ -229,7 +253,7 @@ static BwdWs bwd_ws(void* ws, int B, int Hq, int Tq, int d) {
   BwdWs w;
   w.dq_acc = reinterpret_cast<float*>(ws);
   w.Dv = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + round256((size_t)B * Tq * Hq * d * 4));
-  w.lse2 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(w.Dv) + round256((size_t)B * Hq * Tq * 4));
+  w.lse2 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(w.Dv) + round256((size_t)B * Hq * tq_pad(Tq) * 4));
   return w;
 }
 
@@ -256,15 +280,16 @@ int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void
   if ((st = check_ws(ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d))) return st;
   if ((st = device_setup())) return st;
   const BwdWs w = bwd_ws(ws, B, Hq, Tq, d);
-  const long long threads = (long long)B * Tq * Hq * (d / 8);
+  const int Tp = tq_pad(Tq);
+  const long long threads = std::max((long long)B * Tq * Hq * (d / 8), (long long)B * Hq * (Tp - Tq));
   const unsigned blocks = (unsigned)((threads + 255) / 256);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const __nv_bfloat16* o16 = reinterpret_cast<const __nv_bfloat16*>(o);
   const __nv_bfloat16* do16 = reinterpret_cast<const __nv_bfloat16*>(dO);
   if (d == 64)
-    fa_bwd_preprocess_kernel<64><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, w.dq_acc, B, Hq, Tq);
+    fa_bwd_preprocess_kernel<64><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, w.dq_acc, B, Hq, Tq, Tp);
   else
-    fa_bwd_preprocess_kernel<128><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, w.dq_acc, B, Hq, Tq);
+    fa_bwd_preprocess_kernel<128><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, w.dq_acc, B, Hq, Tq, Tp);
   return launch_status();
 }
 
@@ -295,11 +320,16 @@ int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO
   p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
   p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tq = Tq; p.Tk = Tk; p.causal = causal;
+  p.Tq_pad = tq_pad(Tq);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_kv_tiles = (Tk + 127) / 128;
+  p.n_items = p.n_kv_tiles * B * Hkv;
   p.wait_limit_ns = kWaitLimitNs;
-  dim3 grid(p.n_kv_tiles, B * Hkv);
+  // One CTA per item (the kernel also runs persistently over a smaller grid;
+  // measured slower here because an item's K/V reload then waits on the
+  // previous item's last MMAs).
+  dim3 grid(p.n_items);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64)
     fa_bwd_dkdv_kernel<64><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);

@@ -37,11 +37,14 @@ namespace fa {
 // ---------------------------------------------------------------------------
 // preprocess
 // ---------------------------------------------------------------------------
+// Dv and lse2 rows have a pitch of Tq_pad = Tq rounded up to 128, so that
+// every 128-row slice starts 16-byte aligned for a bulk copy; the padding
+// entries hold D = 0 and LSE2 = +inf (P = 0).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ Dv, float* __restrict__ lse2,
-    float* __restrict__ dq_acc, int B, int Hq, int Tq) {
+    float* __restrict__ dq_acc, int B, int Hq, int Tq, int Tq_pad) {
   constexpr int LPR = D / 8;  // lanes per row, 8 elements (16 bytes) each
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = gid / LPR;            // row index in [B][Tq][Hq] order
@@ -71,10 +74,17 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(
     const long long bt = row / Hq;
     const int t = (int)(bt % Tq);
     const int b = (int)(bt / Tq);
-    const long long idx = ((long long)b * Hq + h) * Tq + t;
-    Dv[idx] = dot;
-    const float l = lse[idx];
-    lse2[idx] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+    const long long bh = (long long)b * Hq + h;
+    Dv[bh * Tq_pad + t] = dot;
+    const float l = lse[bh * Tq + t];
+    lse2[bh * Tq_pad + t] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+  }
+  const int npad = Tq_pad - Tq;
+  if (npad > 0 && gid < (long long)B * Hq * npad) {
+    const long long bh = gid / npad;
+    const long long idx = bh * Tq_pad + Tq + gid % npad;
+    Dv[idx] = 0.f;
+    lse2[idx] = INFINITY;
   }
 }
 
@@ -111,8 +121,10 @@ struct BwdParams {
   __nv_bfloat16* dk;   // [B][Tk][Hkv][d]
   __nv_bfloat16* dv;
   int B, Hq, Hkv, Tq, Tk, causal;
+  int Tq_pad;          // row pitch of lse2 / Dv
   float scale, scale_log2;
   int n_kv_tiles;
+  int n_items;         // n_kv_tiles * B * Hkv
   unsigned long long wait_limit_ns;
 };
 
@@ -142,24 +154,29 @@ struct BwdCfg {
   static constexpr int NBOX = D / 64;
   static constexpr int BOX_BYTES = 128 * 128;
   static constexpr int TILE = NBOX * BOX_BYTES;         // 128 rows x D bf16
-  // d = 64: two S^T buffers in tensor memory and dQ leaves through a shared-
-  // memory tile and a bulk tensor reduce.  d = 128: one S^T buffer (tensor
-  // memory is full) and dQ leaves through vector reductions.
+  // d = 64: two S^T buffers in tensor memory, two K/V buffers in shared
+  // memory (the next item's K/V load overlaps this item) and dQ leaves
+  // through a shared-memory tile and a bulk tensor reduce.  d = 128: one of
+  // each (tensor and shared memory are full) and dQ leaves through vector
+  // reductions.
   static constexpr int NSBUF = (D == 64) ? 2 : 1;
+  static constexpr int NKV = (D == 64) ? 2 : 1;
   static constexpr bool DQ_TMA = (D == 64);
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = TILE;
-  static constexpr int OFF_Q = 2 * TILE;                // 2 stages
-  static constexpr int OFF_DO = 4 * TILE;               // 2 stages
-  static constexpr int OFF_DS = 6 * TILE;               // 128 x 128 bf16, 2 boxes
-  static constexpr int OFF_DQS = OFF_DS + 2 * BOX_BYTES;  // fp32 128 x D staging (DQ_TMA only)
-  static constexpr int DQS_BYTES = DQ_TMA ? 128 * D * 4 : 0;
-  static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;   // [2][128] f32
-  static constexpr int OFF_DD = OFF_LSE + 2 * 128 * 4;  // [2][128] f32
-  static constexpr int OFF_BAR = OFF_DD + 2 * 128 * 4;
-  // kv_full, qdo_full[2], qdo_empty[2], s_full[2], p_full[2], dp_full, ds_full,
-  // dq_full[2], dq_free[2], dkdv_done, mma_done
-  static constexpr int NBAR = 17;
+  static constexpr int NQ = (D == 64) ? 3 : 2;          // Q / dO / LSE2 / D stages
+  static constexpr int OFF_K = 0;                       // NKV buffers of (K, V)
+  static constexpr int OFF_Q = 2 * NKV * TILE;          // NQ stages
+  static constexpr int OFF_DO = OFF_Q + NQ * TILE;      // NQ stages
+  static constexpr int OFF_DS = OFF_DO + NQ * TILE;     // 128 x 128 bf16, 2 boxes
+  // fp32 staging of 32 dQ columns (one 128-byte swizzled box), reused for
+  // each box of the tile (DQ_TMA only)
+  static constexpr int OFF_DQS = OFF_DS + 2 * BOX_BYTES;
+  static constexpr int DQS_BYTES = DQ_TMA ? 128 * 32 * 4 : 0;
+  static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;   // [NQ][128] f32
+  static constexpr int OFF_DD = OFF_LSE + NQ * 128 * 4; // [NQ][128] f32
+  static constexpr int OFF_BAR = OFF_DD + NQ * 128 * 4;
+  // kv_full[2], kv_empty[2], qdo_full[3], qdo_empty[3], s_full[2], p_full[2],
+  // dp_full, ds_full, dq_full[2], dq_free[2], dkdv_done, mma_done
+  static constexpr int NBAR = 22;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int THREADS = 448;                   // 3 warpgroups + MMA warp + TMA warp
@@ -172,7 +189,35 @@ struct BwdCfg {
   static constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 1, 1);
   static_assert(TM_DP + 128 <= TMEM_COLS, "tensor memory overflow");
+  static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+  static_assert(NQ <= 3, "barrier slots");
 };
+
+// One work item: the 128-key tile kt of KV head hkv of batch b, against
+// every query tile (of every query head of the GQA group) that sees it.
+struct BwdItem {
+  int b, hkv, j0, qt_begin, nq, n_it;
+};
+
+__device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
+  BwdItem it;
+  // Key tiles of one (batch, KV head) are adjacent in item order, so the
+  // head's dQ accumulator rows and Q/dO tiles stay in L2 while they run.
+  const int kt = item % p.n_kv_tiles;
+  const int hb = item / p.n_kv_tiles;
+  it.b = hb / p.Hkv;
+  it.hkv = hb % p.Hkv;
+  it.j0 = kt * 128;
+  const int n_qt = (p.Tq + 127) / 128;
+  it.qt_begin = 0;
+  if (p.causal) {
+    const int qmin = it.j0 - (p.Tk - p.Tq);   // first query that sees key j0
+    it.qt_begin = qmin <= 0 ? 0 : min(n_qt, qmin / 128);
+  }
+  it.nq = n_qt - it.qt_begin;
+  it.n_it = (p.Hq / p.Hkv) * it.nq;
+  return it;
+}
 
 template <int D>
 __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
@@ -184,48 +229,42 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
     return;
   }
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  const uint32_t bar_kv = bar0;
-  auto bar_qdo_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto bar_qdo_empty = [&](int s) { return bar0 + 8u * (3 + s); };
-  auto bar_s_full = [&](int b) { return bar0 + 8u * (5 + b); };
-  auto bar_p_full = [&](int b) { return bar0 + 8u * (7 + b); };
-  const uint32_t bar_dp_full = bar0 + 8u * 9;
-  const uint32_t bar_ds_full = bar0 + 8u * 10;
-  auto bar_dq_full = [&](int b) { return bar0 + 8u * (11 + b); };
-  auto bar_dq_free = [&](int b) { return bar0 + 8u * (13 + b); };
-  const uint32_t bar_dkdv_done = bar0 + 8u * 15;
-  const uint32_t bar_mma_done = bar0 + 8u * 16;
+  auto bar_kv_full = [&](int k) { return bar0 + 8u * k; };
+  auto bar_kv_empty = [&](int k) { return bar0 + 8u * (2 + k); };
+  auto bar_qdo_full = [&](int s) { return bar0 + 8u * (4 + s); };
+  auto bar_qdo_empty = [&](int s) { return bar0 + 8u * (7 + s); };
+  auto bar_s_full = [&](int b) { return bar0 + 8u * (10 + b); };
+  auto bar_p_full = [&](int b) { return bar0 + 8u * (12 + b); };
+  const uint32_t bar_dp_full = bar0 + 8u * 14;
+  const uint32_t bar_ds_full = bar0 + 8u * 15;
+  auto bar_dq_full = [&](int b) { return bar0 + 8u * (16 + b); };
+  auto bar_dq_free = [&](int b) { return bar0 + 8u * (18 + b); };
+  const uint32_t bar_dkdv_done = bar0 + 8u * 20;
+  const uint32_t bar_mma_done = bar0 + 8u * 21;
+  // Q/dO stage of global iteration g and the parity of its use of that stage.
+  auto stg = [&](int g) { return g % C::NQ; };
+  auto stg_par = [&](int g) { return (uint32_t)((g / C::NQ) & 1); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
   float* dd_s = reinterpret_cast<float*>(smem + C::OFF_DD);
+  auto aK = [&](int kvb) { return sbase + C::OFF_K + (2 * kvb) * C::TILE; };
+  auto aV = [&](int kvb) { return sbase + C::OFF_K + (2 * kvb + 1) * C::TILE; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Key tiles of one (batch, KV head) are adjacent in launch order, so the
-  // head's dQ accumulator rows and Q/dO tiles stay in L2 while they run.
-  const int kt = blockIdx.x;
-  const int hb = blockIdx.y;
-  const int b = hb / p.Hkv;
-  const int hkv = hb % p.Hkv;
-  const int j0 = kt * 128;
   const int G = p.Hq / p.Hkv;
-  const int n_qt = (p.Tq + 127) / 128;
-  int qt_begin = 0;
-  if (p.causal) {
-    const int qmin = j0 - (p.Tk - p.Tq);     // first query that sees key j0
-    qt_begin = qmin <= 0 ? 0 : min(n_qt, qmin / 128);
-  }
-  const int nq = n_qt - qt_begin;
-  const int n_it = G * nq;
   WaitCtl wc{abort_flag, p.wait_limit_ns};
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(bar_kv, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_qdo_full(s), 32);
+    for (int s = 0; s < C::NQ; ++s) {
+      mbar_init(bar_qdo_full(s), 1);
       mbar_init(bar_qdo_empty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_kv_full(s), 1);
+      mbar_init(bar_kv_empty(s), 1);
       mbar_init(bar_s_full(s), 1);
       mbar_init(bar_p_full(s), 128);
       mbar_init(bar_dq_full(s), 1);
@@ -245,210 +284,251 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  auto it_head = [&](int it) { return hkv * G + it / nq; };
-  auto it_q0 = [&](int it) { return (qt_begin + it % nq) * 128; };
 
   if (warp == 13) {
     // ------------------------------------------------------------ producer
-    bool ok = true;
-    int issued = 0;
-    if (n_it > 0) {
-      if (lane == 0) {
-        tma_prefetch_desc(&p.tm_q);
-        tma_prefetch_desc(&p.tm_do);
-        tma_prefetch_desc(&p.tm_k);
-        tma_prefetch_desc(&p.tm_v);
-        mbar_arrive_expect_tx(bar_kv, 2 * C::TILE);
-        for (int kb = 0; kb < C::NBOX; ++kb) {
-          tma_load_4d(sbase + C::OFF_K + kb * C::BOX_BYTES, &p.tm_k, bar_kv, kb * 64, hkv, j0, b);
-          tma_load_4d(sbase + C::OFF_V + kb * C::BOX_BYTES, &p.tm_v, bar_kv, kb * 64, hkv, j0, b);
-        }
-      }
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int s = it & 1;
-        const int h = it_head(it);
-        const int q0 = it_q0(it);
-        if (it >= 2) ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_empty(s), ((it >> 1) - 1) & 1, wc));
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_do);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      bool ok = true;
+      int gi = 0, ki = 0, issued_kv = 0;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const BwdItem I = bwd_item(p, item);
+        if (I.n_it == 0) continue;
+        const int kvb = ki % C::NKV;
+        if (ki >= C::NKV) ok = mbar_wait(bar_kv_empty(kvb), ((ki / C::NKV) - 1) & 1, wc);
         if (!ok) break;
-        const size_t rbase = ((size_t)b * p.Hq + h) * p.Tq;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = lane * 4 + e;
-          const int q = q0 + r;
-          lse_s[s * 128 + r] = q < p.Tq ? p.lse2[rbase + q] : INFINITY;
-          dd_s[s * 128 + r] = q < p.Tq ? p.Dv[rbase + q] : 0.f;
+        mbar_arrive_expect_tx(bar_kv_full(kvb), 2 * C::TILE);
+        for (int kb = 0; kb < C::NBOX; ++kb) {
+          tma_load_4d(aK(kvb) + kb * C::BOX_BYTES, &p.tm_k, bar_kv_full(kvb), kb * 64, I.hkv, I.j0, I.b);
+          tma_load_4d(aV(kvb) + kb * C::BOX_BYTES, &p.tm_v, bar_kv_full(kvb), kb * 64, I.hkv, I.j0, I.b);
         }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar_qdo_full(s), 2 * C::TILE);
+        ++issued_kv;
+        for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
+          const int s = stg(gi);
+          const int h = I.hkv * G + it / I.nq;
+          const int q0 = (I.qt_begin + it % I.nq) * 128;
+          if (gi >= C::NQ) ok = mbar_wait(bar_qdo_empty(s), stg_par(gi) ^ 1u, wc);
+          if (!ok) break;
+          const size_t rbase = ((size_t)I.b * p.Hq + h) * p.Tq_pad + q0;
+          mbar_arrive_expect_tx(bar_qdo_full(s), 2 * C::TILE + 2 * 512);
           for (int kb = 0; kb < C::NBOX; ++kb) {
-            tma_load_4d(sbase + C::OFF_Q + s * C::TILE + kb * C::BOX_BYTES, &p.tm_q, bar_qdo_full(s),
-                        kb * 64, h, q0, b);
-            tma_load_4d(sbase + C::OFF_DO + s * C::TILE + kb * C::BOX_BYTES, &p.tm_do, bar_qdo_full(s),
-                        kb * 64, h, q0, b);
+            tma_load_4d(sbase + C::OFF_Q + s * C::TILE + kb * C::BOX_BYTES, &p.tm_q, bar_qdo_full(s), kb * 64, h,
+                        q0, I.b);
+            tma_load_4d(sbase + C::OFF_DO + s * C::TILE + kb * C::BOX_BYTES, &p.tm_do, bar_qdo_full(s), kb * 64,
+                        h, q0, I.b);
           }
-        } else {
-          mbar_arrive(bar_qdo_full(s));
+          bulk_load(sbase + C::OFF_LSE + s * 512, p.lse2 + rbase, 512, bar_qdo_full(s));
+          bulk_load(sbase + C::OFF_DD + s * 512, p.Dv + rbase, 512, bar_qdo_full(s));
         }
-        ++issued;
+        ++ki;
       }
-      if (!ok && lane == 0) {
-        mbar_wait_drain(bar_kv, 0, p.wait_limit_ns);
-        for (int it = max(0, issued - 2); it < issued; ++it)
-          mbar_wait_drain(bar_qdo_full(it & 1), (it >> 1) & 1, p.wait_limit_ns);
+      if (!ok) {
+        for (int k = max(0, issued_kv - C::NKV); k < issued_kv; ++k)
+          mbar_wait_drain(bar_kv_full(k % C::NKV), (k / C::NKV) & 1, p.wait_limit_ns);
+        for (int g = max(0, gi - C::NQ); g <= gi; ++g)
+          mbar_wait_drain(bar_qdo_full(stg(g)), stg_par(g), p.wait_limit_ns);
       }
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_it > 0) {
+    if (lane == 0) {
       const uint32_t tDP = tmem + C::TM_DP, tDV = tmem + C::TM_DV, tDK = tmem + C::TM_DK;
       auto tS = [&](int buf) { return tmem + C::TM_S0 + 128 * buf; };
-      const uint32_t aK = sbase + C::OFF_K, aV = sbase + C::OFF_V, aDS = sbase + C::OFF_DS;
-      auto aQ = [&](int it) { return sbase + C::OFF_Q + (it & 1) * C::TILE; };
-      auto aDO = [&](int it) { return sbase + C::OFF_DO + (it & 1) * C::TILE; };
+      const uint32_t aDS = sbase + C::OFF_DS;
+      auto aQ = [&](int g) { return sbase + C::OFF_Q + stg(g) * C::TILE; };
+      auto aDO = [&](int g) { return sbase + C::OFF_DO + stg(g) * C::TILE; };
       auto kdesc = [&](uint32_t base, int k) {  // K-major tile, k-th 16-element slice of d
         return smem_desc_sw128(base + (k >> 2) * C::BOX_BYTES + (k & 3) * 32, 16, 1024);
       };
       auto mndesc = [&](uint32_t base, int k) {  // MN-major view, k-th 16-row slice
         return smem_desc_sw128(base + k * 16 * 128, C::BOX_BYTES, 1024);
       };
-      auto issue_s = [&](int it) {
-        const int buf = it % C::NSBUF;
+      auto issue_s = [&](int g, int kvb) {
+        const int buf = g % C::NSBUF;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss(tS(buf), kdesc(aK, k), kdesc(aQ(it), k), C::IDESC_SS, k > 0);
+        for (int k = 0; k < D / 16; ++k) mma_ss(tS(buf), kdesc(aK(kvb), k), kdesc(aQ(g), k), C::IDESC_SS, k > 0);
         mma_commit(bar_s_full(buf));
       };
-      auto issue_dp = [&](int it) {
+      auto issue_dp = [&](int g, int kvb) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc(aV, k), kdesc(aDO(it), k), C::IDESC_SS, k > 0);
+        for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc(aV(kvb), k), kdesc(aDO(g), k), C::IDESC_SS, k > 0);
         mma_commit(bar_dp_full);
       };
-      bool ok = mbar_wait(bar_kv, 0, wc);
-      if (ok) ok = mbar_wait(bar_qdo_full(0), 0, wc);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-        issue_dp(0);
-      }
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int buf = it % C::NSBUF;
-        if (C::NSBUF == 2 && it + 1 < n_it) {
-          // S^T of the next tile into the other buffer, which dQ(it-1) used.
-          ok = mbar_wait(bar_qdo_full((it + 1) & 1), ((it + 1) >> 1) & 1, wc);
-          if (ok && it >= 1) ok = mbar_wait(bar_dq_free((it + 1) & 1), ((it - 1) >> 1) & 1, wc);
+      bool ok = true;
+      int gi = 0, ki = 0;
+      bool started = false;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const BwdItem I = bwd_item(p, item);
+        if (I.n_it == 0) continue;
+        const int kvb = ki % C::NKV;
+        if (!started) {
+          ok = mbar_wait(bar_kv_full(kvb), (ki / C::NKV) & 1, wc);
+          if (ok) ok = mbar_wait(bar_qdo_full(stg(0)), stg_par(0), wc);
           if (!ok) break;
           tc_fence_after();
-          issue_s(it + 1);
+          issue_s(0, kvb);
+          issue_dp(0, kvb);
+          started = true;
         }
-        ok = mbar_wait(bar_p_full(buf), (it / C::NSBUF) & 1, wc);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_ts(tDV, tS(buf) + k * 8, mndesc(aDO(it), k), C::IDESC_TS, it > 0 || k > 0);
-        ok = mbar_wait(bar_ds_full, it & 1, wc);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_ts(tDK, tDP + k * 8, mndesc(aQ(it), k), C::IDESC_TS, it > 0 || k > 0);
-        mma_commit(bar_qdo_empty(it & 1));
-        // dQ(it) = dS K into the S^T buffer of this tile (P^T consumed above).
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mma_ss(tS(buf), mndesc(aDS, k), mndesc(aK, k), C::IDESC_DQ, k > 0);
-        mma_commit(bar_dq_full(buf));
-        if (it + 1 < n_it) {
-          if (C::NSBUF == 1) {
-            ok = mbar_wait(bar_qdo_full((it + 1) & 1), ((it + 1) >> 1) & 1, wc);
+        const bool has_next_item = item + (int)gridDim.x < p.n_items;
+        for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
+          const int buf = gi % C::NSBUF;
+          const bool last = it + 1 == I.n_it;
+          const bool has_next = !last || has_next_item;
+          // K/V buffer of the next iteration; waits for it when it belongs
+          // to the next item.
+          const int kvb_next = last ? (ki + 1) % C::NKV : kvb;
+          auto wait_next_operands = [&]() -> bool {
+            if (!mbar_wait(bar_qdo_full(stg(gi + 1)), stg_par(gi + 1), wc)) return false;
+            if (last && !mbar_wait(bar_kv_full(kvb_next), ((ki + 1) / C::NKV) & 1, wc)) return false;
+            return true;
+          };
+          if (C::NSBUF == 2 && has_next) {
+            // S^T of the next iteration into the other buffer, which dQ of
+            // the previous iteration used.
+            ok = wait_next_operands();
+            if (ok && gi >= 1) ok = mbar_wait(bar_dq_free((gi + 1) & 1), ((gi - 1) >> 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
+            issue_s(gi + 1, kvb_next);
           }
-          issue_dp(it + 1);
-          if (C::NSBUF == 1) {
-            ok = mbar_wait(bar_dq_free(0), it & 1, wc);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(it + 1);
+          ok = mbar_wait(bar_p_full(buf), (gi / C::NSBUF) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_ts(tDV, tS(buf) + k * 8, mndesc(aDO(gi), k), C::IDESC_TS, it > 0 || k > 0);
+          ok = mbar_wait(bar_ds_full, gi & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_ts(tDK, tDP + k * 8, mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
+          mma_commit(bar_qdo_empty(stg(gi)));
+          // dQ = dS K into this iteration's S^T buffer (P^T consumed above).
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mma_ss(tS(buf), mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
+          mma_commit(bar_dq_full(buf));
+          if (last) {
+            mma_commit(bar_kv_empty(kvb));
+            mma_commit(bar_dkdv_done);
+          }
+          if (has_next) {
+            if (C::NSBUF == 1) {
+              ok = wait_next_operands();
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_dp(gi + 1, kvb_next);
+            if (C::NSBUF == 1) {
+              ok = mbar_wait(bar_dq_free(0), gi & 1, wc);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(gi + 1, kvb_next);
+            }
           }
         }
+        ++ki;
       }
-      if (ok) mma_commit(bar_dkdv_done);
       mma_commit(bar_mma_done);
       mbar_wait_drain(bar_mma_done, 0, p.wait_limit_ns);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ P^T (WG-A)
     const int j = threadIdx.x;               // key row in the tile == TMEM lane
-    const int key = j0 + j;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int qmin = key - (p.Tk - p.Tq);    // causal: first query that sees this key
-    const bool key_ok = key < p.Tk;
     const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int s = it & 1, buf = it % C::NSBUF;
-      const int q0 = it_q0(it);
-      const uint32_t tS = tmem + C::TM_S0 + 128 * buf + lane_off;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), (it >> 1) & 1, wc));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(buf), (it / C::NSBUF) & 1, wc));
-      if (!ok) break;
-      tc_fence_after();
-      const float* lrow = lse_s + s * 128;
-      const int cmin = p.causal ? qmin - q0 : 0;  // columns < cmin are masked
+    int gi = 0, ki = 0;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const BwdItem I = bwd_item(p, item);
+      const int key = I.j0 + j;
+      const int qmin = key - (p.Tk - p.Tq);  // causal: first query that sees this key
+      const bool key_ok = key < p.Tk;
+      for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
+        const int s = stg(gi), buf = gi % C::NSBUF;
+        const int q0 = (I.qt_begin + it % I.nq) * 128;
+        const uint32_t tS = tmem + C::TM_S0 + 128 * buf + lane_off;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), stg_par(gi), wc));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(buf), (gi / C::NSBUF) & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+        const float* lrow = lse_s + s * 128;
+        const int cmin = p.causal ? qmin - q0 : 0;  // columns < cmin are masked
+        const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > 0);
+        uint32_t sv[2][32];
+        tmem_ld32(tS, sv[0]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int col = c * 32 + 2 * e;
-          const float2 l2 = *reinterpret_cast<const float2*>(lrow + col);
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
-                                      sl2, make_float2(-l2.x, -l2.y));
-          float p0 = ex2_approx(x.x);
-          float p1 = ex2_approx(x.y);
-          if (!key_ok || col < cmin) p0 = 0.f;
-          if (!key_ok || col + 1 < cmin) p1 = 0.f;
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + c * 16, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p_full(buf));
-    }
-    // ------------------------------------------------------------ dK, dV out
-    if (n_it > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dkdv_done, 0, wc));
-    tc_fence_after();
-    const bool have = n_it > 0 && ok;
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off;
-      const float mul = which ? p.scale : 1.f;
-      __nv_bfloat16* dst = (which ? p.dk : p.dv) + (((size_t)b * p.Tk + (key < p.Tk ? key : 0)) * p.Hkv + hkv) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        if (have) {
-          tmem_ld32(tsrc + c * 32, v);
+        for (int c = 0; c < 4; ++c) {
           tmem_wait_ld();
-        } else {
+          if (c + 1 < 4) tmem_ld32(tS + (c + 1) * 32, sv[(c + 1) & 1]);
+          const uint32_t* cur = sv[c & 1];
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
+          for (int e = 0; e < 16; ++e) {
+            const int col = c * 32 + 2 * e;
+            const float2 l2 = *reinterpret_cast<const float2*>(lrow + col);
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(cur[2 * e]), __uint_as_float(cur[2 * e + 1])),
+                                        sl2, make_float2(-l2.x, -l2.y));
+            float p0 = ex2_approx(x.x);
+            float p1 = ex2_approx(x.y);
+            if (masked) {
+              if (!key_ok || col < cmin) p0 = 0.f;
+              if (!key_ok || col + 1 < cmin) p1 = 0.f;
+            }
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          // The next chunk's load reads columns >= 32*(c+1); this store
+          // writes columns 16*c .. 16*c+15, already consumed.
+          tmem_st16(tS + c * 16, pk);
         }
-        uint4 pk[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p_full(buf));
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- dK, dV out
+      const bool have = I.n_it > 0;
+      if (have) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_dkdv_done, ki & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+      }
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pw[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
-        if (key < p.Tk) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off;
+        const float mul = which ? p.scale : 1.f;
+        __nv_bfloat16* dst =
+            (which ? p.dk : p.dv) + (((size_t)I.b * p.Tk + (key < p.Tk ? key : 0)) * p.Hkv + I.hkv) * D;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (have) {
+            tmem_ld32(tsrc + c * 32, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          uint4 pk[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pw[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+          if (key < p.Tk) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+          }
         }
       }
+      // dK/dV have been read: the next item's first dV/dK MMAs (which
+      // overwrite them) wait for this warpgroup's next p_full arrival.
+      tc_fence_before();
+      if (have) ++ki;
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ dS (WG-B)
@@ -457,104 +537,121 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
     const uint32_t tDP = tmem + C::TM_DP + lane_off;
     uint8_t* ds_row = smem + C::OFF_DS + j * 128;
     bool ok = true;
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int s = it & 1, buf = it % C::NSBUF;
-      const uint32_t tP = tmem + C::TM_S0 + 128 * buf + lane_off;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), (it >> 1) & 1, wc));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_p_full(buf), (it / C::NSBUF) & 1, wc));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, it & 1, wc));
-      if (!ok) break;
-      tc_fence_after();
-      const float* drow = dd_s + s * 128;
+    int gi = 0;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const BwdItem I = bwd_item(p, item);
+      for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
+        const int s = stg(gi), buf = gi % C::NSBUF;
+        const uint32_t tP = tmem + C::TM_S0 + 128 * buf + lane_off;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), stg_par(gi), wc));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_p_full(buf), (gi / C::NSBUF) & 1, wc));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, gi & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+        const float* drow = dd_s + s * 128;
+        uint32_t pp[2][16], dp[2][32];
+        tmem_ld16(tP, pp[0]);
+        tmem_ld32(tDP, dp[0]);
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t pp[16], dp[32];
-        tmem_ld16(tP + c4 * 16, pp);
-        tmem_ld32(tDP + c4 * 32, dp);
-        tmem_wait_ld();
-        uint32_t ds[16];
+        for (int c4 = 0; c4 < 4; ++c4) {
+          tmem_wait_ld();
+          const uint32_t* cp = pp[c4 & 1];
+          const uint32_t* cd = dp[c4 & 1];
+          uint32_t ds[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[e]));
-          const float2 dd = *reinterpret_cast<const float2*>(drow + c4 * 32 + 2 * e);
-          const float2 t = __fadd2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
-                                      make_float2(-dd.x, -dd.y));
-          const float2 r = __fmul2_rn(pf, t);
-          ds[e] = pack_bf16x2(r.x, r.y);
+          for (int e = 0; e < 16; ++e) {
+            const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cp[e]));
+            const float2 dd = *reinterpret_cast<const float2*>(drow + c4 * 32 + 2 * e);
+            const float2 t = __fadd2_rn(make_float2(__uint_as_float(cd[2 * e]), __uint_as_float(cd[2 * e + 1])),
+                                        make_float2(-dd.x, -dd.y));
+            const float2 r = __fmul2_rn(pf, t);
+            ds[e] = pack_bf16x2(r.x, r.y);
+          }
+          // The next chunk's loads read columns at or beyond 32*(c4+1); the
+          // store below writes columns 16*c4 .. 16*c4+15, already consumed.
+          if (c4 + 1 < 4) {
+            tmem_ld16(tP + (c4 + 1) * 16, pp[(c4 + 1) & 1]);
+            tmem_ld32(tDP + (c4 + 1) * 32, dp[(c4 + 1) & 1]);
+          }
+          tmem_st16(tDP + c4 * 16, ds);
+          // dS into shared memory: row j of box (c4/2), 16-byte chunks
+          // 4*(c4%2) .. +3, 128-byte swizzle (chunk ^ (row % 8)).
+          uint8_t* box = ds_row + (c4 >> 1) * C::BOX_BYTES;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int chunk = 4 * (c4 & 1) + cc;
+            *reinterpret_cast<uint4*>(box + ((chunk ^ (j & 7)) << 4)) =
+                make_uint4(ds[4 * cc], ds[4 * cc + 1], ds[4 * cc + 2], ds[4 * cc + 3]);
+          }
         }
-        tmem_st16(tDP + c4 * 16, ds);
-        // dS into shared memory: row j of box (c4/2), 16-byte chunks
-        // 4*(c4%2) .. +3, 128-byte swizzle (chunk ^ (row % 8)).
-        uint8_t* box = ds_row + (c4 >> 1) * C::BOX_BYTES;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int chunk = 4 * (c4 & 1) + cc;
-          *reinterpret_cast<uint4*>(box + ((chunk ^ (j & 7)) << 4)) =
-              make_uint4(ds[4 * cc], ds[4 * cc + 1], ds[4 * cc + 2], ds[4 * cc + 3]);
-        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar_ds_full);
       }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_ds_full);
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------ dQ (WG-C)
     const int r = threadIdx.x - 256;         // query row in the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     bool ok = true;
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int buf = it % C::NSBUF;
-      const int h = it_head(it);
-      const int q0 = it_q0(it);
-      const uint32_t tDQ = tmem + C::TM_S0 + 128 * buf + lane_off;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_dq_full(buf), (it / C::NSBUF) & 1, wc));
-      if (!ok) break;
-      tc_fence_after();
-      if constexpr (C::DQ_TMA) {
-        uint32_t v[D];
+    int gi = 0;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const BwdItem I = bwd_item(p, item);
+      for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
+        const int buf = gi % C::NSBUF;
+        const int h = I.hkv * G + it / I.nq;
+        const int q0 = (I.qt_begin + it % I.nq) * 128;
+        const uint32_t tDQ = tmem + C::TM_S0 + 128 * buf + lane_off;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_dq_full(buf), (gi / C::NSBUF) & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+        if constexpr (C::DQ_TMA) {
+          uint32_t v[D];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(tDQ + c * 32, v + c * 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar_dq_free(buf));
-        // The previous tile's bulk reduce must have read the staging tile.
-        if (threadIdx.x == 256) bulk_wait_group_read0();
-        named_bar_sync(2, 128);
-        // fp32 staging, boxes of 32 columns, 128-byte swizzle.
-#pragma unroll
-        for (int c = 0; c < D / 4; ++c) {
-          const int box = c >> 3, chunk = c & 7;
-          *reinterpret_cast<float4*>(smem + C::OFF_DQS + box * (128 * 128) + r * 128 + ((chunk ^ (r & 7)) << 4)) =
-              make_float4(__uint_as_float(v[4 * c]) * p.scale, __uint_as_float(v[4 * c + 1]) * p.scale,
-                          __uint_as_float(v[4 * c + 2]) * p.scale, __uint_as_float(v[4 * c + 3]) * p.scale);
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(2, 128);
-        if (threadIdx.x == 256) {
-#pragma unroll
-          for (int box = 0; box < D / 32; ++box)
-            tma_reduce_add_4d(&p.tm_dq, sbase + C::OFF_DQS + box * (128 * 128), box * 32, h, q0, b);
-          bulk_commit_group();
-        }
-      } else {
-        const int q = q0 + r;
-        float* dst = p.dq_acc + (((size_t)b * p.Tq + (q < p.Tq ? q : 0)) * p.Hq + h) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tDQ + c * 32, v);
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(tDQ + c * 32, v + c * 32);
           tmem_wait_ld();
-          if (q < p.Tq) {
+          tc_fence_before();
+          mbar_arrive(bar_dq_free(buf));
+          // fp32 staging, one 32-column box at a time (128-byte swizzle);
+          // before each refill the previous bulk reduce must have read it.
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
-                         __uint_as_float(v[4 * e + 1]) * p.scale, __uint_as_float(v[4 * e + 2]) * p.scale,
-                         __uint_as_float(v[4 * e + 3]) * p.scale);
+          for (int box = 0; box < D / 32; ++box) {
+            if (threadIdx.x == 256) bulk_wait_group_read0();
+            named_bar_sync(2, 128);
+#pragma unroll
+            for (int chunk = 0; chunk < 8; ++chunk) {
+              const int c = box * 8 + chunk;
+              *reinterpret_cast<float4*>(smem + C::OFF_DQS + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+                  make_float4(__uint_as_float(v[4 * c]) * p.scale, __uint_as_float(v[4 * c + 1]) * p.scale,
+                              __uint_as_float(v[4 * c + 2]) * p.scale, __uint_as_float(v[4 * c + 3]) * p.scale);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(2, 128);
+            if (threadIdx.x == 256) {
+              tma_reduce_add_4d(&p.tm_dq, sbase + C::OFF_DQS, box * 32, h, q0, I.b);
+              bulk_commit_group();
+            }
           }
+        } else {
+          const int q = q0 + r;
+          float* dst = p.dq_acc + (((size_t)I.b * p.Tq + (q < p.Tq ? q : 0)) * p.Hq + h) * D;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tDQ + c * 32, v);
+            tmem_wait_ld();
+            if (q < p.Tq) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
+                           __uint_as_float(v[4 * e + 1]) * p.scale, __uint_as_float(v[4 * e + 2]) * p.scale,
+                           __uint_as_float(v[4 * e + 3]) * p.scale);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar_dq_free(buf));
         }
-        tc_fence_before();
-        mbar_arrive(bar_dq_free(buf));
       }
     }
     if constexpr (C::DQ_TMA) {

@@ -8,9 +8,14 @@
 // Masks Still Apply"; "FlashAttention" (interview track), "Softmax without
 // seeing the whole row" (keep m and l as one log-sum-exp per row).
 //
-// B200 mapping (one CTA = two 128-row query tiles of one (batch, head)):
-//   warp 9      TMA producer: Q0, Q1 once, then K_j, V_j tiles into a ring of
-//               shared-memory stages (128-byte swizzle, 64-column boxes).
+// B200 mapping.  The kernel is persistent: one CTA per SM walks a list of
+// work items, each two 128-row query tiles of one (batch, head), so that one
+// item's set-up (Q load, first K/V tiles) and epilogue overlap the next
+// item's MMAs instead of leaving the SM idle.
+//   warp 9      TMA producer: Q0, Q1 of each item into one of two Q buffers,
+//               then K_j, V_j tiles into a ring of shared-memory stages
+//               (128-byte swizzle, 64-column boxes), running ahead across
+//               items.
 //   warp 8      MMA issuer (one thread): S_w = Q_w K_j^T into tensor memory,
 //               O_w += P_w V_j with P_w read from tensor memory.
 //   warps 0-3   softmax for query tile 0 (TMEM lanes 0..127, one row per
@@ -41,7 +46,8 @@ struct FwdParams {
   int B, Hq, Hkv, Tq, Tk;
   int causal;
   float scale_log2;   // scale * log2(e)
-  int n_mblocks;      // ceil(Tq / 256)
+  int n_mblocks;      // ceil(Tq / 256): work items per (batch, head)
+  int n_items;        // B * Hq * n_mblocks
   unsigned long long wait_limit_ns;
 };
 
@@ -52,13 +58,13 @@ struct FwdCfg {
   static constexpr int NBOX = D / 64;            // 64-element swizzle boxes along d
   static constexpr int BOX_BYTES = 128 * 128;    // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;
-  static constexpr int NSTAGE = (D == 64) ? 8 : 4;
-  static constexpr int OFF_Q0 = 0;
-  static constexpr int OFF_Q1 = TILE_BYTES;
-  static constexpr int OFF_RING = 2 * TILE_BYTES;
+  static constexpr int NSTAGE = (D == 64) ? 6 : 3;
+  static constexpr int OFF_Q = 0;                // 2 buffers x (Q0, Q1)
+  static constexpr int OFF_RING = 4 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSTAGE * TILE_BYTES;
-  // barriers: q_full, kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2], p_full[2], o_final[2], mma_done
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+  // q_full[2], q_empty[2], kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2],
+  // p_full[2], o_final[2], mma_done
+  static constexpr int NBAR = 4 + 2 * NSTAGE + 2 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 320;
@@ -66,7 +72,35 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
   static constexpr float RESCALE_THRESHOLD = 8.0f;
+  static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
 };
+
+// One work item: two query tiles [m0, m0 + 256) of head h of batch b.
+struct FwdItem {
+  int b, h, hkv, m0, n_kv;
+};
+
+template <int D>
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
+  using C = FwdCfg<D>;
+  FwdItem it;
+  // Query blocks of one (batch, head) are adjacent in item order, so they
+  // share that head's K/V tiles through L2; within a head the heaviest
+  // causal block (the last one) comes first.
+  const int bh = item / p.n_mblocks;
+  it.b = bh / p.Hq;
+  it.h = bh % p.Hq;
+  it.hkv = it.h / (p.Hq / p.Hkv);
+  it.m0 = (p.n_mblocks - 1 - item % p.n_mblocks) * 2 * C::BM;
+  const int n_kv_all = (p.Tk + C::BN - 1) / C::BN;
+  it.n_kv = n_kv_all;
+  if (p.causal) {
+    const int last_row = min(it.m0 + 2 * C::BM, p.Tq) - 1;
+    const int kmax = last_row + (p.Tk - p.Tq);  // last visible key (inclusive)
+    it.n_kv = kmax < 0 ? 0 : min(n_kv_all, kmax / C::BN + 1);
+  }
+  return it;
+}
 
 template <int D>
 __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
@@ -75,42 +109,29 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar_base = sbase + C::OFF_BAR;
-  auto bar_q = [&]() { return bar_base; };
-  auto bar_kv_full = [&](int s) { return bar_base + 8u * (1 + s); };
-  auto bar_kv_empty = [&](int s) { return bar_base + 8u * (1 + C::NSTAGE + s); };
-  auto bar_s_full = [&](int w) { return bar_base + 8u * (1 + 2 * C::NSTAGE + w); };
-  auto bar_p_full = [&](int w) { return bar_base + 8u * (3 + 2 * C::NSTAGE + w); };
-  auto bar_o_final = [&](int w) { return bar_base + 8u * (5 + 2 * C::NSTAGE + w); };
-  const uint32_t bar_mma_done = bar_base + 8u * (7 + 2 * C::NSTAGE);
+  auto bar_q_full = [&](int q) { return bar_base + 8u * q; };
+  auto bar_q_empty = [&](int q) { return bar_base + 8u * (2 + q); };
+  auto bar_kv_full = [&](int s) { return bar_base + 8u * (4 + s); };
+  auto bar_kv_empty = [&](int s) { return bar_base + 8u * (4 + C::NSTAGE + s); };
+  auto bar_s_full = [&](int w) { return bar_base + 8u * (4 + 2 * C::NSTAGE + w); };
+  auto bar_p_full = [&](int w) { return bar_base + 8u * (6 + 2 * C::NSTAGE + w); };
+  auto bar_o_final = [&](int w) { return bar_base + 8u * (8 + 2 * C::NSTAGE + w); };
+  const uint32_t bar_mma_done = bar_base + 8u * (10 + 2 * C::NSTAGE);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  auto q_addr = [&](int qb, int w) { return sbase + C::OFF_Q + (2 * qb + w) * C::TILE_BYTES; };
+  auto stage_addr = [&](int s) { return sbase + C::OFF_RING + s * C::TILE_BYTES; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Query blocks of one (batch, head) are adjacent in launch order, so they
-  // share that head's K/V tiles through L2; within a head the heaviest
-  // causal block (the last one) goes first.
-  const int bh = blockIdx.y;
-  const int b = bh / p.Hq;
-  const int h = bh % p.Hq;
-  const int hkv = h / (p.Hq / p.Hkv);
-  const int mblock = p.n_mblocks - 1 - (int)blockIdx.x;
-  const int m0 = mblock * 2 * C::BM;
-
-  // Number of KV tiles this CTA visits.
-  const int n_kv_all = (p.Tk + C::BN - 1) / C::BN;
-  int n_kv = n_kv_all;
-  if (p.causal) {
-    const int last_row = min(m0 + 2 * C::BM, p.Tq) - 1;
-    const int kmax = last_row + (p.Tk - p.Tq);  // last visible key (inclusive)
-    n_kv = kmax < 0 ? 0 : min(n_kv_all, kmax / C::BN + 1);
-  }
-
   WaitCtl wc{abort_flag, p.wait_limit_ns};
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(bar_q(), 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(bar_q_full(q), 1);
+      mbar_init(bar_q_empty(q), 1);
+    }
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(bar_kv_full(s), 1);
       mbar_init(bar_kv_empty(s), 1);
@@ -134,100 +155,113 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
 
   if (warp == 9) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_kv > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
-      mbar_arrive_expect_tx(bar_q(), 2 * C::TILE_BYTES);
-      for (int kb = 0; kb < C::NBOX; ++kb) {
-        tma_load_4d(sbase + C::OFF_Q0 + kb * C::BOX_BYTES, &p.tm_q, bar_q(), kb * 64, h, m0, b);
-        tma_load_4d(sbase + C::OFF_Q1 + kb * C::BOX_BYTES, &p.tm_q, bar_q(), kb * 64, h, m0 + C::BM, b);
-      }
-      int issued = 0;
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        for (int which = 0; which < 2 && ok; ++which) {
-          const int idx = 2 * j + which;
-          const int s = idx % C::NSTAGE;
-          const int round = idx / C::NSTAGE;
-          if (round > 0) ok = mbar_wait(bar_kv_empty(s), (round - 1) & 1, wc);
-          if (!ok) break;
-          mbar_arrive_expect_tx(bar_kv_full(s), C::TILE_BYTES);
-          const CUtensorMap* tm = which ? &p.tm_v : &p.tm_k;
-          for (int kb = 0; kb < C::NBOX; ++kb)
-            tma_load_4d(sbase + C::OFF_RING + s * C::TILE_BYTES + kb * C::BOX_BYTES, tm,
-                        bar_kv_full(s), kb * 64, hkv, j * C::BN, b);
-          ++issued;
+      int qi = 0;         // items with work, in this CTA's order
+      int idx = 0;        // K/V ring slot counter
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const FwdItem it = fwd_item<D>(p, item);
+        if (it.n_kv == 0) continue;
+        const int qb = qi & 1;
+        if (qi >= 2) ok = mbar_wait(bar_q_empty(qb), ((qi >> 1) - 1) & 1, wc);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_q_full(qb), 2 * C::TILE_BYTES);
+        for (int kb = 0; kb < C::NBOX; ++kb) {
+          tma_load_4d(q_addr(qb, 0) + kb * C::BOX_BYTES, &p.tm_q, bar_q_full(qb), kb * 64, it.h, it.m0, it.b);
+          tma_load_4d(q_addr(qb, 1) + kb * C::BOX_BYTES, &p.tm_q, bar_q_full(qb), kb * 64, it.h, it.m0 + C::BM, it.b);
         }
+        for (int j = 0; j < it.n_kv && ok; ++j) {
+          for (int which = 0; which < 2 && ok; ++which, ++idx) {
+            const int s = idx % C::NSTAGE;
+            const int round = idx / C::NSTAGE;
+            if (round > 0) ok = mbar_wait(bar_kv_empty(s), (round - 1) & 1, wc);
+            if (!ok) break;
+            mbar_arrive_expect_tx(bar_kv_full(s), C::TILE_BYTES);
+            const CUtensorMap* tm = which ? &p.tm_v : &p.tm_k;
+            for (int kb = 0; kb < C::NBOX; ++kb)
+              tma_load_4d(stage_addr(s) + kb * C::BOX_BYTES, tm, bar_kv_full(s), kb * 64, it.hkv, j * C::BN, it.b);
+          }
+        }
+        ++qi;
       }
       if (!ok) {
         // Let every copy already issued land before the CTA can exit.
-        mbar_wait_drain(bar_q(), 0, p.wait_limit_ns);
-        for (int idx = max(0, issued - C::NSTAGE); idx < issued; ++idx)
-          mbar_wait_drain(bar_kv_full(idx % C::NSTAGE), (idx / C::NSTAGE) & 1, p.wait_limit_ns);
+        for (int q = max(0, qi - 1); q <= qi; ++q) mbar_wait_drain(bar_q_full(q & 1), (q >> 1) & 1, p.wait_limit_ns);
+        for (int k = max(0, idx - C::NSTAGE); k < idx; ++k)
+          mbar_wait_drain(bar_kv_full(k % C::NSTAGE), (k / C::NSTAGE) & 1, p.wait_limit_ns);
       }
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_kv > 0) {
+    if (lane == 0) {
       const uint32_t tS[2] = {tmem, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
-      const uint32_t q_addr[2] = {sbase + C::OFF_Q0, sbase + C::OFF_Q1};
-      auto stage_addr = [&](int s) { return sbase + C::OFF_RING + s * C::TILE_BYTES; };
-      auto issue_s = [&](int w, int sK) {
+      auto issue_s = [&](int w, uint32_t qa, int sK) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;
-          mma_ss(tS[w], smem_desc_sw128(q_addr[w] + off, 16, 1024),
-                 smem_desc_sw128(stage_addr(sK) + off, 16, 1024), C::IDESC_S, k > 0);
+          mma_ss(tS[w], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(stage_addr(sK) + off, 16, 1024),
+                 C::IDESC_S, k > 0);
         }
       };
       auto issue_pv = [&](int w, int sV, bool first) {
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k) {
-          mma_ts(tO[w], tS[w] + k * 8,
-                 smem_desc_sw128(stage_addr(sV) + k * 16 * 128, C::BOX_BYTES, 1024), C::IDESC_O,
+          mma_ts(tO[w], tS[w] + k * 8, smem_desc_sw128(stage_addr(sV) + k * 16 * 128, C::BOX_BYTES, 1024), C::IDESC_O,
                  (!first) || k > 0);
         }
       };
-      bool ok = mbar_wait(bar_q(), 0, wc);
-      tc_fence_after();
-      int sV_prev = 0;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int iK = 2 * j, iV = 2 * j + 1;
-        const int sK = iK % C::NSTAGE, sV = iV % C::NSTAGE;
-        ok = mbar_wait(bar_kv_full(sK), (iK / C::NSTAGE) & 1, wc);
+      bool ok = true;
+      int qi = 0, g = 0;  // items with work, global KV tile counter
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const FwdItem it = fwd_item<D>(p, item);
+        if (it.n_kv == 0) continue;
+        const int qb = qi & 1;
+        ok = mbar_wait(bar_q_full(qb), (qi >> 1) & 1, wc);
         if (!ok) break;
         tc_fence_after();
-        issue_s(0, sK);
-        mma_commit(bar_s_full(0));
-        if (j > 0) {
-          ok = mbar_wait(bar_p_full(1), (j - 1) & 1, wc);
+        int sV_prev = 0;
+        for (int j = 0; j < it.n_kv && ok; ++j) {
+          const int gt = g + j;
+          const int iK = 2 * gt, iV = 2 * gt + 1;
+          const int sK = iK % C::NSTAGE, sV = iV % C::NSTAGE;
+          ok = mbar_wait(bar_kv_full(sK), (iK / C::NSTAGE) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(1, sV_prev, j - 1 == 0);
-          mma_commit(bar_kv_empty(sV_prev));
+          issue_s(0, q_addr(qb, 0), sK);
+          mma_commit(bar_s_full(0));
+          if (j > 0) {
+            ok = mbar_wait(bar_p_full(1), (gt - 1) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(1, sV_prev, j - 1 == 0);
+            mma_commit(bar_kv_empty(sV_prev));
+          }
+          issue_s(1, q_addr(qb, 1), sK);
+          mma_commit(bar_s_full(1));
+          mma_commit(bar_kv_empty(sK));
+          ok = mbar_wait(bar_p_full(0), gt & 1, wc);
+          if (!ok) break;
+          ok = mbar_wait(bar_kv_full(sV), (iV / C::NSTAGE) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(0, sV, j == 0);
+          sV_prev = sV;
         }
-        issue_s(1, sK);
-        mma_commit(bar_s_full(1));
-        mma_commit(bar_kv_empty(sK));
-        ok = mbar_wait(bar_p_full(0), j & 1, wc);
         if (!ok) break;
-        ok = mbar_wait(bar_kv_full(sV), (iV / C::NSTAGE) & 1, wc);
+        mma_commit(bar_o_final(0));
+        ok = mbar_wait(bar_p_full(1), (g + it.n_kv - 1) & 1, wc);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(0, sV, j == 0);
-        sV_prev = sV;
-      }
-      if (ok) {
-        mma_commit(bar_o_final(0));
-        ok = mbar_wait(bar_p_full(1), (n_kv - 1) & 1, wc);
-        if (ok) {
-          tc_fence_after();
-          issue_pv(1, sV_prev, n_kv - 1 == 0);
-          mma_commit(bar_kv_empty(sV_prev));
-          mma_commit(bar_o_final(1));
-        }
+        issue_pv(1, sV_prev, it.n_kv - 1 == 0);
+        mma_commit(bar_kv_empty(sV_prev));
+        mma_commit(bar_o_final(1));
+        mma_commit(bar_q_empty(qb));
+        g += it.n_kv;
+        ++qi;
       }
       // Wait until every MMA issued above has completed before teardown.
       mma_commit(bar_mma_done);
@@ -240,99 +274,123 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + w * 128 + lane_off;
     const uint32_t tO = tmem + 256 + w * D + lane_off;
-    const int row = m0 + w * C::BM + r;
-    const int key_limit = p.causal ? min(p.Tk, row + (p.Tk - p.Tq) + 1) : p.Tk;  // keys < limit visible
-    float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
-    float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(w), j & 1, wc));
+    int qi = 0, g = 0;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const FwdItem it = fwd_item<D>(p, item);
+      const int row = it.m0 + w * C::BM + r;
+      const int key_limit = p.causal ? min(p.Tk, row + (p.Tk - p.Tq) + 1) : p.Tk;  // keys < limit visible
+      float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
+      float l = 0.f;
+      for (int j = 0; j < it.n_kv; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(w), (g + j) & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t su[128];  // S row, then P (bf16 pairs) packed in place
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, su + c * 32);
+        tmem_wait_ld();
+        const int nvalid = key_limit - j * C::BN;
+        if (__any_sync(0xffffffffu, nvalid < C::BN)) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= nvalid) su[c] = __float_as_uint(-INFINITY);
+        }
+        // Row maximum: eight independent chains, then a short tree.
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(su[i]);
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], __uint_as_float(su[c + i]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_tile = mx * p.scale_log2;
+        // Lazy rescale: move the reference only when the maximum grew by more
+        // than the threshold (or there was no reference yet).
+        const bool move = (m_tile > m_ref + C::RESCALE_THRESHOLD) || (m_ref == -INFINITY && m_tile != -INFINITY);
+        float alpha = 1.f;
+        if (move) {
+          alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_tile);
+          m_ref = m_tile;
+          l *= alpha;
+        }
+        const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nref = make_float2(-ref, -ref);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(su[2 * c]), __uint_as_float(su[2 * c + 1])), sl2, nref);
+          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          acc[c & 3] = __fadd2_rn(acc[c & 3], pr);
+          su[c] = pack_bf16x2(pr.x, pr.y);
+        }
+        const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        l += a.x + a.y;
+        tmem_st32(tS, su);
+        tmem_st32(tS + 32, su + 32);
+        if (j > 0 && __any_sync(0xffffffffu, move)) {
+          // O row *= alpha.  The PV of the previous tile has completed: the
+          // commit behind s_full tracks every MMA issued before it, and the
+          // PV of this tile waits for p_full below.
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p_full(w));
+      }
       if (!ok) break;
-      tc_fence_after();
-      uint32_t su[128];  // S row, then P (bf16 pairs) packed in place
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, su + c * 32);
-      tmem_wait_ld();
-      const int nvalid = key_limit - j * C::BN;
-      if (nvalid < C::BN) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= nvalid) su[c] = __float_as_uint(-INFINITY);
+      // ---------------------------------------------------------- epilogue
+      if (it.n_kv > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_final(w), qi & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
       }
-      float mx = __uint_as_float(su[0]);
+      const bool in_range = row < p.Tq;
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.o + (((size_t)it.b * p.Tq + (in_range ? row : 0)) * p.Hq + it.h) * D;
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(su[c]));
-      const float m_tile = mx * p.scale_log2;
-      // Lazy rescale: move the reference only when the maximum grew by more
-      // than the threshold (or there was no reference yet).
-      const bool move = (m_tile > m_ref + C::RESCALE_THRESHOLD) || (m_ref == -INFINITY && m_tile != -INFINITY);
-      float alpha = 1.f;
-      if (move) {
-        alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_tile);
-        m_ref = m_tile;
-        l *= alpha;
-      }
-      const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(su[2 * c]), p.scale_log2, -ref));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(su[2 * c + 1]), p.scale_log2, -ref));
-        sum0 += p0;
-        sum1 += p1;
-        su[c] = pack_bf16x2(p0, p1);
-      }
-      l += sum0 + sum1;
-      tmem_st32(tS, su);
-      tmem_st32(tS + 32, su + 32);
-      if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // O row *= alpha.  The PV of the previous tile has completed: the
-        // commit behind s_full tracks every MMA issued before it, and the
-        // PV of this tile waits for p_full below.
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (it.n_kv > 0) {
           tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
+        } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + c * 32, o);
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint4 packed[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pw[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = packed[i];
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p_full(w));
-    }
-    // ------------------------------------------------------------ epilogue
-    if (ok && n_kv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_final(w), 0, wc));
-    tc_fence_after();
-    const bool in_range = row < p.Tq;
-    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = p.o + (((size_t)b * p.Tq + (in_range ? row : 0)) * p.Hq + h) * D;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32];
-      if (n_kv > 0 && ok) {
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
-      }
-      uint4 packed[4];
-      uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        pw[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
       if (in_range) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = packed[i];
+        const float lse = (l > 0.f) ? (m_ref * 0.69314718055994531f + logf(l)) : -INFINITY;
+        p.lse[((size_t)it.b * p.Hq + it.h) * p.Tq + row] = lse;
       }
-    }
-    if (in_range) {
-      const float lse = (l > 0.f) ? (m_ref * 0.69314718055994531f + logf(l)) : -INFINITY;
-      p.lse[((size_t)b * p.Hq + h) * p.Tq + row] = lse;
+      // O has been read: the next item's first PV (which overwrites O) is
+      // issued only after this warpgroup's next p_full arrival.
+      tc_fence_before();
+      if (it.n_kv > 0) {
+        g += it.n_kv;
+        ++qi;
+      }
     }
   }
 

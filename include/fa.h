@@ -156,6 +156,32 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
                       void* stream);
 
 /*
+ * fa_decode_splitkv_noalloc -- fa_decode_splitkv for callers that cannot
+ * allocate device memory where they call it: code running inside a CUDA
+ * graph capture or a plug-in interface that only hands over inputs and
+ * outputs, or a latency-critical loop that cannot afford cudaMalloc's
+ * implicit device synchronisation.  The pages have no counterpart; this is a
+ * deployment convenience around the same kernels.
+ *   Arguments as for fa_decode_splitkv, without ws/ws_bytes.  The chunk
+ *   partials live in a 32 MiB array inside the library (every GPU that loads
+ *   the library holds it until the process exits), so
+ *   fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk) must be at most
+ *   33554432; larger calls return FA_ERR_WORKSPACE before any launch.
+ *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   The first call on a device looks up the array's device address and sets
+ *   kernel attributes for that device; make that first call outside any
+ *   stream capture.
+ *   All calls share the one array: calls whose kernels overlap on the GPU
+ *   (different streams, or different host threads, without ordering) race
+ *   and produce wrong results.  Calls ordered on one stream are safe; the
+ *   array keeps the last call's contents, which no later call relies on.
+ */
+int fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                              const int* seqlens_k, void* o, float* lse,
+                              int B, int Hq, int Hkv, int Tk_max, int d, float scale, int chunk,
+                              void* stream);
+
+/*
  * fa_check -- synchronise `stream`, then read and clear the device status
  * word that kernels set when a bounded wait expires.  Returns FA_OK,
  * FA_ERR_TIMEOUT, or FA_ERR_CUDA if the synchronisation itself failed.

@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     backward_workspace_bytes,
     check,
     decode_splitkv,
+    decode_splitkv_noalloc,
     decode_workspace_bytes,
     forward,
     load_library,

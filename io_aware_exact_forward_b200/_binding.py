@@ -39,6 +39,7 @@ SIGNATURES = {
     "fa_backward_dq_finalize": (_c_int, [_vp] * 2 + [_c_size] + [_c_int] * 6 + [_vp]),
     "fa_decode_workspace_bytes": (_c_size, [_c_int] * 5),
     "fa_decode_splitkv": (_c_int, [_vp] * 6 + [_vp, _c_size] + [_c_int] * 5 + [_c_float, _c_int, _vp]),
+    "fa_decode_splitkv_noalloc": (_c_int, [_vp] * 6 + [_c_int] * 5 + [_c_float, _c_int, _vp]),
     "fa_check": (_c_int, [_vp]),
     "fa_selftest_bounded_wait": (_c_int, [_c_int, _vp]),
 }
@@ -171,6 +172,27 @@ def decode_splitkv(q, k_cache, v_cache, seqlens, scale=None, chunk=256, workspac
                                _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tk_max, d, float(scale),
                                int(chunk), _stream_ptr(dev))
     _raise("fa_decode_splitkv", st)
+    return out, lse
+
+
+def decode_splitkv_noalloc(q, k_cache, v_cache, seqlens, scale=None, chunk=256, out=None, lse=None):
+    """Split-KV decode through fa_decode_splitkv_noalloc: the chunk partials
+    live in the library's built-in 32 MiB device array instead of a caller
+    workspace.  Calls that overlap on the GPU share that array and race."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    Tk_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+    dev = q.device
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_dev(n, t, torch.bfloat16, dev)
+    _check_dev("seqlens", seqlens, torch.int32, dev)
+    if scale is None:
+        scale = d ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev) if lse is None else lse
+    st = lib.fa_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse),
+                                       B, Hq, Hkv, Tk_max, d, float(scale), int(chunk), _stream_ptr(dev))
+    _raise("fa_decode_splitkv_noalloc", st)
     return out, lse
 
 

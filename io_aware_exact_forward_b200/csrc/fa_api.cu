@@ -478,3 +478,55 @@ extern "C" int fa_selftest_bounded_wait(int limit_us, void* stream) {
       (unsigned long long)limit_us * 1000ull);
   return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// Split-KV decode without caller-provided workspace.
+//
+// For callers that cannot allocate device memory at the call site -- code
+// that runs while a CUDA graph is being captured through an API that
+// forbids allocation, plug-in interfaces that hand over only the input and
+// output tensors, or latency-critical loops where cudaMalloc's implicit
+// device synchronisation is not acceptable.  The chunk partials live in one
+// file-scope device array that every GPU loading this library keeps until
+// the process exits.
+// ---------------------------------------------------------------------------
+namespace fa {
+
+static constexpr size_t kDecodeScratchBytes = 32u << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+// Device address of g_decode_scratch for the current device, looked up once
+// per device (host code may not use the symbol itself as an address).
+static int decode_scratch_ptr(void** out) {
+  static void* cache[kMaxDevices];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return FA_ERR_CUDA;
+    cache[dev] = ptr;
+  }
+  *out = cache[dev];
+  return FA_OK;
+}
+
+}  // namespace fa
+
+extern "C" int fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                         const int* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv,
+                                         int Tk_max, int d, float scale, int chunk, void* stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Tk_max < 0 || chunk < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // The partials of this call must fit in the built-in scratch array.
+  if (fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk) > kDecodeScratchBytes) return FA_ERR_WORKSPACE;
+  if (B == 0) return FA_OK;
+  void* scratch = nullptr;
+  const int st = decode_scratch_ptr(&scratch);
+  if (st) return st;
+  // Every partial the combine step reads is written first by the split step
+  // of the same call, so nothing in the scratch needs clearing.
+  return fa_decode_splitkv(q, k_cache, v_cache, seqlens_k, o, lse, scratch, kDecodeScratchBytes, B, Hq, Hkv,
+                           Tk_max, d, scale, chunk, stream);
+}

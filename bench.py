@@ -45,11 +45,13 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["fa", "reference"], default="fa")
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4])
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (smaller cases for profiler captures only)")
     return ap.parse_args()
 
 
@@ -216,6 +218,9 @@ def cpu_baseline(w, inp_cpu, budget_s):
 def run_reference(args, w, rank):
     if rank != 0:
         return 0
+    if w.decode:
+        print(json.dumps({"impl": "reference", "unavailable": "reference arm covers the prefill workloads"}))
+        return 0
     from workloads import prefill_inputs
     inp = prefill_inputs(w.with_(B=1), device="cpu")
     heads = [(0, h) for h in range(w.Hq)]
@@ -239,6 +244,26 @@ def run_reference(args, w, rank):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------------------
+# timing helpers shared by every rank
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(value, dist, device=None):
+    """Largest `value` over all ranks (the job's time is the slowest rank's)."""
+    if dist is None:
+        return value
+    import torch
+    dev = device if (device is not None and dist.get_backend() == "nccl") else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(work_per_rank_step, world, steps, elapsed_ms):
+    """Whole-job rate: every rank's work over the slowest rank's time."""
+    return world * work_per_rank_step * steps / (elapsed_ms * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -319,16 +344,11 @@ def run_fa(args, w, rank, world, dist):
     status = lib.fa_check(sp)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
-    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     seg = [sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps for i in range(4)]
-    if dist is not None:
-        import torch.distributed as tdist
-        t = torch.tensor([elapsed_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
     ms_per_step = elapsed_ms / args.steps
     f_fwd, f_bwd = flops(w)
-    value = world * (f_fwd + f_bwd) * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_rate(f_fwd + f_bwd, world, args.steps, elapsed_ms) / 1e12
 
     # roofline of the dominant kernel (largest share of the step)
     peaks = load_peaks()
@@ -385,13 +405,8 @@ def run_fa(args, w, rank, world, dist):
             e2e_step()
         e1.record(stream)
         barrier()
-        e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            import torch.distributed as tdist
-            t = torch.tensor([e_ms], device=dev)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * (f_fwd + f_bwd) * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        e2e = {"value": job_rate(f_fwd + f_bwd, world, args.e2e_steps, e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "ms_per_step": e_ms / args.e2e_steps}
 
@@ -422,10 +437,90 @@ def run_fa(args, w, rank, world, dist):
     return 0
 
 
+def run_decode(args, w, rank, world, dist):
+    """Split-KV decode of the B=64, Hq=32, Hkv=8, d=128 batch: one step is
+    fa_decode_splitkv (split kernel + combine kernel); value is algorithmic
+    HBM GB/s (K and V of every cached token read once, plus q, o, lse)."""
+    import ctypes
+    import torch
+    import io_aware_exact_forward_b200 as fa
+    from workloads import decode_inputs
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = fa.load_library()
+    inp = decode_inputs(w, device=dev, seed=w.seed + rank)
+    q, kc, vc, sl = inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"]
+    B, Hq, Hkv, Tk_max, d, chunk = w.B, w.Hq, w.Hkv, w.T, w.d, w.chunk
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    wsb = lib.fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    P = ctypes.c_void_p
+    stream = torch.cuda.current_stream(dev)
+    sp = P(stream.cuda_stream)
+    args_c = (P(q.data_ptr()), P(kc.data_ptr()), P(vc.data_ptr()), P(sl.data_ptr()), P(o.data_ptr()),
+              P(lse.data_ptr()), P(ws.data_ptr()), wsb, B, Hq, Hkv, Tk_max, d, w.scale, chunk, sp)
+
+    def step():
+        st = lib.fa_decode_splitkv(*args_c)
+        if st != 0:
+            raise RuntimeError(f"fa_decode_splitkv: {fa.STATUS.get(st, st)}")
+
+    total_keys = int(sl.sum().item())
+    alg_bytes = total_keys * Hkv * d * 2 * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    # the cache (2 x 4.3 GB) is far larger than L2: no flush needed
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    gpu_index = local
+    with ClockSampler(gpu_index) as clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        barrier()
+    if lib.fa_check(sp) != 0:
+        raise RuntimeError("device status set during the timed region")
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    value = job_rate(alg_bytes, world, args.steps, ms) / 1e9
+    peaks = load_peaks()
+    # dominant kernel time: split kernel alone, timed separately on the same stream
+    if rank == 0:
+        line = {
+            "metric": "split-KV decode HBM GB/s (bf16 KV cache, 1xB200) and % of HBM peak",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "Tk_max": Tk_max, "d": d, "chunk": chunk,
+                       "total_cached_tokens": total_keys, "l2": "KV cache larger than L2", "seed": w.seed},
+            "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_combine_kernel", "bound": "hbm",
+                         "achieved": value / world, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": value / world / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy",
+                         "traffic": traffic_from_profile("fa_decode_split_kernel", w.name),
+                         "algorithmic_per_launch": alg_bytes},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     from workloads import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = w.with_(B=args.batch)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     dist = None
@@ -439,6 +534,8 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
     try:
+        if w.decode:
+            return run_decode(args, w, rank, world, dist)
         return run_fa(args, w, rank, world, dist)
     finally:
         if dist is not None:

@@ -13,21 +13,26 @@
 //                shared memory; the CTA walks the query tiles of every query
 //                head of its GQA group.  Per tile, in tensor memory:
 //                  S^T = K Q^T, dP^T = V dO^T          (SS MMAs)
-//                  P^T = 2^{S^T*scale*log2e - LSE2}   (compute warps, bf16
-//                        written over S^T)
+//                  P^T = 2^{S^T*scale*log2e - LSE2}   (P warps, bf16 into
+//                        half of the S^T columns)
 //                  dV += P^T dO                         (TS MMA)
-//                  dS^T = P^T * (dP^T - D)             (compute warps, bf16
-//                        over dP^T and into shared memory as the A operand)
+//                  dS^T = P^T * (dP^T - D)             (dS warps, bf16 into
+//                        the other half of the S^T columns, and dS into
+//                        shared memory as an A operand)
 //                  dK += dS^T Q                         (TS MMA)
 //                  dQ_tile = dS K                       (SS MMA)
+//                The next tile's dP^T MMA is issued as soon as the dS warps
+//                have read this tile's dP^T.
 //                dQ_tile is read by a second warpgroup and added into an fp32
 //                accumulator in global memory with vector reductions (every
 //                KV tile contributes to every query row it sees).  dK and dV
 //                are summed over the group's heads in tensor memory, so the
 //                GQA sum needs no atomics.
 //   dq_convert   dq = bf16(accumulator).
-// Warp roles in dkdv: 0-3 compute (one key row per thread = TMEM lane),
-// 4-7 dQ reduction (one query row per thread), 8 MMA issuer, 9 TMA producer.
+// Warp roles in dkdv: 0-7 P^T and 8-15 dS (two warps per TMEM lane quarter,
+// one per half of the 128 query columns, so that one warp computes while the
+// other waits for its tensor-memory loads), 16-19 dQ reduction (one query
+// row per thread), 20 MMA issuer, 21 TMA producer.
 #pragma once
 
 #include "fa_ptx.cuh"
@@ -175,11 +180,15 @@ struct BwdCfg {
   static constexpr int OFF_DD = OFF_LSE + NQ * 128 * 4; // [NQ][128] f32
   static constexpr int OFF_BAR = OFF_DD + NQ * 128 * 4;
   // kv_full[2], kv_empty[2], qdo_full[3], qdo_empty[3], s_full[2], p_full[2],
-  // dp_full, ds_full, dq_full[2], dq_free[2], dkdv_done, mma_done
-  static constexpr int NBAR = 22;
+  // dp_full, ds_full, dq_full[2], dq_free[2], dkdv_done, mma_done, dp_free
+  static constexpr int NBAR = 23;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
-  static constexpr int THREADS = 448;                   // 3 warpgroups + MMA warp + TMA warp
+  // warps 0-7 P^T (two per TMEM lane quarter, one per half of the query
+  // columns), 8-15 dS, 16-19 dQ, 20 MMA issuer, 21 TMA producer
+  static constexpr int THREADS = 704;
+  static constexpr int MMA_WARP = 20;
+  static constexpr int LOAD_WARP = 21;
   static constexpr int TMEM_COLS = 512;
   static constexpr int TM_DV = 0;
   static constexpr int TM_DK = D;
@@ -220,7 +229,7 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -241,6 +250,7 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
   auto bar_dq_free = [&](int b) { return bar0 + 8u * (18 + b); };
   const uint32_t bar_dkdv_done = bar0 + 8u * 20;
   const uint32_t bar_mma_done = bar0 + 8u * 21;
+  const uint32_t bar_dp_free = bar0 + 8u * 22;
   // Q/dO stage of global iteration g and the parity of its use of that stage.
   auto stg = [&](int g) { return g % C::NQ; };
   auto stg_par = [&](int g) { return (uint32_t)((g / C::NQ) & 1); };
@@ -266,17 +276,18 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
       mbar_init(bar_kv_full(s), 1);
       mbar_init(bar_kv_empty(s), 1);
       mbar_init(bar_s_full(s), 1);
-      mbar_init(bar_p_full(s), 128);
+      mbar_init(bar_p_full(s), 256);
       mbar_init(bar_dq_full(s), 1);
       mbar_init(bar_dq_free(s), 128);
     }
     mbar_init(bar_dp_full, 1);
-    mbar_init(bar_ds_full, 128);
+    mbar_init(bar_dp_free, 256);
+    mbar_init(bar_ds_full, 256);
     mbar_init(bar_dkdv_done, 1);
     mbar_init(bar_mma_done, 1);
     fence_barrier_init();
   }
-  if (warp == 12) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -285,7 +296,7 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 13) {
+  if (warp == C::LOAD_WARP) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -332,7 +343,7 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
           mbar_wait_drain(bar_qdo_full(stg(g)), stg_par(g), p.wait_limit_ns);
       }
     }
-  } else if (warp == 12) {
+  } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t tDP = tmem + C::TM_DP, tDV = tmem + C::TM_DV, tDK = tmem + C::TM_DK;
@@ -395,20 +406,31 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
             tc_fence_after();
             issue_s(gi + 1, kvb_next);
           }
+          // P^T of query half h sits in columns [64h, 64h+32) of the S^T
+          // buffer, dS^T of that half in [64h+32, 64h+64).
+          auto p_col = [](int k) { return (k < 4) ? k * 8 : 64 + (k - 4) * 8; };
           ok = mbar_wait(bar_p_full(buf), (gi / C::NSBUF) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_ts(tDV, tS(buf) + k * 8, mndesc(aDO(gi), k), C::IDESC_TS, it > 0 || k > 0);
+            mma_ts(tDV, tS(buf) + p_col(k), mndesc(aDO(gi), k), C::IDESC_TS, it > 0 || k > 0);
+          if (has_next) {
+            // dP^T of the next tile as soon as the dS warps have read this one.
+            ok = mbar_wait(bar_dp_free, gi & 1, wc);
+            if (ok && C::NSBUF == 1) ok = wait_next_operands();
+            if (!ok) break;
+            tc_fence_after();
+            issue_dp(gi + 1, kvb_next);
+          }
           ok = mbar_wait(bar_ds_full, gi & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_ts(tDK, tDP + k * 8, mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
+            mma_ts(tDK, tS(buf) + 32 + p_col(k), mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
           mma_commit(bar_qdo_empty(stg(gi)));
-          // dQ = dS K into this iteration's S^T buffer (P^T consumed above).
+          // dQ = dS K into this tile's S^T buffer (P^T and dS^T read above).
 #pragma unroll
           for (int k = 0; k < 8; ++k) mma_ss(tS(buf), mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
           mma_commit(bar_dq_full(buf));
@@ -416,19 +438,11 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
             mma_commit(bar_kv_empty(kvb));
             mma_commit(bar_dkdv_done);
           }
-          if (has_next) {
-            if (C::NSBUF == 1) {
-              ok = wait_next_operands();
-              if (!ok) break;
-              tc_fence_after();
-            }
-            issue_dp(gi + 1, kvb_next);
-            if (C::NSBUF == 1) {
-              ok = mbar_wait(bar_dq_free(0), gi & 1, wc);
-              if (!ok) break;
-              tc_fence_after();
-              issue_s(gi + 1, kvb_next);
-            }
+          if (C::NSBUF == 1 && has_next) {
+            ok = mbar_wait(bar_dq_free(0), gi & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(gi + 1, kvb_next);
           }
         }
         ++ki;
@@ -436,10 +450,11 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
       mma_commit(bar_mma_done);
       mbar_wait_drain(bar_mma_done, 0, p.wait_limit_ns);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P^T (WG-A)
-    const int j = threadIdx.x;               // key row in the tile == TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int lq = warp & 3, half = warp >> 2;  // TMEM lane quarter, query half
+    const int j = lq * 32 + lane;               // key row in the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(lq * 32) << 16;
     const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
     int gi = 0, ki = 0;
@@ -451,25 +466,28 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
       for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
         const int s = stg(gi), buf = gi % C::NSBUF;
         const int q0 = (I.qt_begin + it % I.nq) * 128;
-        const uint32_t tS = tmem + C::TM_S0 + 128 * buf + lane_off;
+        const uint32_t tS = tmem + C::TM_S0 + 128 * buf + lane_off + 64 * half;
         ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), stg_par(gi), wc));
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(buf), (gi / C::NSBUF) & 1, wc));
         if (!ok) break;
         tc_fence_after();
-        const float* lrow = lse_s + s * 128;
-        const int cmin = p.causal ? qmin - q0 : 0;  // columns < cmin are masked
+        const float* lrow = lse_s + s * 128 + 64 * half;
+        const int cmin = p.causal ? qmin - q0 - 64 * half : 0;  // columns < cmin are masked
         const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > 0);
-        uint32_t sv[2][32];
-        tmem_ld32(tS, sv[0]);
+        // 64 query columns in four 16-column chunks; the load of chunk c+1
+        // overlaps the exponentials of chunk c.  P^T (bf16 pairs) goes to
+        // the first 32 columns of this warp's 64, never ahead of its loads.
+        uint32_t sv[2][16];
+        tmem_ld16(tS, sv[0]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           tmem_wait_ld();
-          if (c + 1 < 4) tmem_ld32(tS + (c + 1) * 32, sv[(c + 1) & 1]);
+          if (c + 1 < 4) tmem_ld16(tS + (c + 1) * 16, sv[(c + 1) & 1]);
           const uint32_t* cur = sv[c & 1];
-          uint32_t pk[16];
+          uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int col = c * 32 + 2 * e;
+          for (int e = 0; e < 8; ++e) {
+            const int col = c * 16 + 2 * e;
             const float2 l2 = *reinterpret_cast<const float2*>(lrow + col);
             const float2 x = __ffma2_rn(make_float2(__uint_as_float(cur[2 * e]), __uint_as_float(cur[2 * e + 1])),
                                         sl2, make_float2(-l2.x, -l2.y));
@@ -481,9 +499,7 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
             }
             pk[e] = pack_bf16x2(p0, p1);
           }
-          // The next chunk's load reads columns >= 32*(c+1); this store
-          // writes columns 16*c .. 16*c+15, already consumed.
-          tmem_st16(tS + c * 16, pk);
+          tmem_st8(tS + c * 8, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -499,12 +515,12 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
       }
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off;
+        const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off + half * (D / 2);
         const float mul = which ? p.scale : 1.f;
-        __nv_bfloat16* dst =
-            (which ? p.dk : p.dv) + (((size_t)I.b * p.Tk + (key < p.Tk ? key : 0)) * p.Hkv + I.hkv) * D;
+        __nv_bfloat16* dst = (which ? p.dk : p.dv) +
+                             (((size_t)I.b * p.Tk + (key < p.Tk ? key : 0)) * p.Hkv + I.hkv) * D + half * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t v[32];
           if (have) {
             tmem_ld32(tsrc + c * 32, v);
@@ -526,73 +542,86 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
         }
       }
       // dK/dV have been read: the next item's first dV/dK MMAs (which
-      // overwrite them) wait for this warpgroup's next p_full arrival.
+      // overwrite them) wait for this warp's next p_full arrival.
       tc_fence_before();
       if (have) ++ki;
     }
-  } else if (warp < 8) {
+  } else if (warp < 16) {
     // ------------------------------------------------------------ dS (WG-B)
-    const int j = threadIdx.x - 128;         // key row == TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tDP = tmem + C::TM_DP + lane_off;
-    uint8_t* ds_row = smem + C::OFF_DS + j * 128;
+    const int w8 = warp - 8;
+    const int lq = w8 & 3, half = w8 >> 2;
+    const int j = lq * 32 + lane;               // key row == TMEM lane
+    const uint32_t lane_off = (uint32_t)(lq * 32) << 16;
+    const uint32_t tDP = tmem + C::TM_DP + lane_off + 64 * half;
+    uint8_t* ds_row = smem + C::OFF_DS + half * C::BOX_BYTES + j * 128;
     bool ok = true;
     int gi = 0;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const BwdItem I = bwd_item(p, item);
       for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
         const int s = stg(gi), buf = gi % C::NSBUF;
-        const uint32_t tP = tmem + C::TM_S0 + 128 * buf + lane_off;
+        const uint32_t tP = tmem + C::TM_S0 + 128 * buf + lane_off + 64 * half;  // P^T, then dS^T at +32
         ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), stg_par(gi), wc));
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_p_full(buf), (gi / C::NSBUF) & 1, wc));
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, gi & 1, wc));
         if (!ok) break;
         tc_fence_after();
-        const float* drow = dd_s + s * 128;
-        uint32_t pp[2][16], dp[2][32];
-        tmem_ld16(tP, pp[0]);
-        tmem_ld32(tDP, dp[0]);
+        const float* drow = dd_s + s * 128 + 64 * half;
+        uint32_t pp[2][8], dp[2][16];
+        tmem_ld8(tP, pp[0]);
+        tmem_ld16(tDP, dp[0]);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c = 0; c < 4; ++c) {
           tmem_wait_ld();
-          const uint32_t* cp = pp[c4 & 1];
-          const uint32_t* cd = dp[c4 & 1];
-          uint32_t ds[16];
+          if (c + 1 < 4) {
+            tmem_ld8(tP + (c + 1) * 8, pp[(c + 1) & 1]);
+            tmem_ld16(tDP + (c + 1) * 16, dp[(c + 1) & 1]);
+          } else {
+            // every dP^T column of this warp has been read
+            tc_fence_before();
+            mbar_arrive(bar_dp_free);
+          }
+          const uint32_t* cp = pp[c & 1];
+          const uint32_t* cd = dp[c & 1];
+          uint32_t ds[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
+          for (int e = 0; e < 8; ++e) {
             const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cp[e]));
-            const float2 dd = *reinterpret_cast<const float2*>(drow + c4 * 32 + 2 * e);
+            const float2 dd = *reinterpret_cast<const float2*>(drow + c * 16 + 2 * e);
             const float2 t = __fadd2_rn(make_float2(__uint_as_float(cd[2 * e]), __uint_as_float(cd[2 * e + 1])),
                                         make_float2(-dd.x, -dd.y));
             const float2 r = __fmul2_rn(pf, t);
             ds[e] = pack_bf16x2(r.x, r.y);
           }
-          // The next chunk's loads read columns at or beyond 32*(c4+1); the
-          // store below writes columns 16*c4 .. 16*c4+15, already consumed.
-          if (c4 + 1 < 4) {
-            tmem_ld16(tP + (c4 + 1) * 16, pp[(c4 + 1) & 1]);
-            tmem_ld32(tDP + (c4 + 1) * 32, dp[(c4 + 1) & 1]);
+          tmem_st8(tP + 32 + c * 8, ds);
+          if (c == 0 && gi > 0) {
+            // The shared dS tile is still the A operand of the previous
+            // tile's dQ MMA until that MMA completes (this tile's dP^T can
+            // complete before it).
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
+            if (!ok) break;
           }
-          tmem_st16(tDP + c4 * 16, ds);
-          // dS into shared memory: row j of box (c4/2), 16-byte chunks
-          // 4*(c4%2) .. +3, 128-byte swizzle (chunk ^ (row % 8)).
-          uint8_t* box = ds_row + (c4 >> 1) * C::BOX_BYTES;
+          // dS into shared memory: row j of box `half`, 16-byte chunks 2c and
+          // 2c+1, 128-byte swizzle (chunk ^ (row % 8)).
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int chunk = 4 * (c4 & 1) + cc;
-            *reinterpret_cast<uint4*>(box + ((chunk ^ (j & 7)) << 4)) =
+          for (int cc = 0; cc < 2; ++cc) {
+            const int chunk = 2 * c + cc;
+            *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (j & 7)) << 4)) =
                 make_uint4(ds[4 * cc], ds[4 * cc + 1], ds[4 * cc + 2], ds[4 * cc + 3]);
           }
         }
+        if (!ok) break;
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar_ds_full);
       }
     }
-  } else if (warp < 12) {
+  } else if (warp < 20) {
     // ------------------------------------------------------------ dQ (WG-C)
-    const int r = threadIdx.x - 256;         // query row in the tile == TMEM lane
+    const int r = threadIdx.x - 512;         // query row in the tile == TMEM lane
+    const int lead = 512;                    // thread that issues the bulk reduces
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     bool ok = true;
     int gi = 0;
@@ -607,28 +636,29 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
         if (!ok) break;
         tc_fence_after();
         if constexpr (C::DQ_TMA) {
-          uint32_t v[D];
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) tmem_ld32(tDQ + c * 32, v + c * 32);
+          uint32_t v[2][32];
+          tmem_ld32(tDQ, v[0]);
+          tmem_ld32(tDQ + 32, v[1]);
           tmem_wait_ld();
           tc_fence_before();
           mbar_arrive(bar_dq_free(buf));
           // fp32 staging, one 32-column box at a time (128-byte swizzle);
           // before each refill the previous bulk reduce must have read it.
 #pragma unroll
-          for (int box = 0; box < D / 32; ++box) {
-            if (threadIdx.x == 256) bulk_wait_group_read0();
+          for (int box = 0; box < 2; ++box) {
+            if (threadIdx.x == lead) bulk_wait_group_read0();
             named_bar_sync(2, 128);
 #pragma unroll
             for (int chunk = 0; chunk < 8; ++chunk) {
-              const int c = box * 8 + chunk;
               *reinterpret_cast<float4*>(smem + C::OFF_DQS + r * 128 + ((chunk ^ (r & 7)) << 4)) =
-                  make_float4(__uint_as_float(v[4 * c]) * p.scale, __uint_as_float(v[4 * c + 1]) * p.scale,
-                              __uint_as_float(v[4 * c + 2]) * p.scale, __uint_as_float(v[4 * c + 3]) * p.scale);
+                  make_float4(__uint_as_float(v[box][4 * chunk]) * p.scale,
+                              __uint_as_float(v[box][4 * chunk + 1]) * p.scale,
+                              __uint_as_float(v[box][4 * chunk + 2]) * p.scale,
+                              __uint_as_float(v[box][4 * chunk + 3]) * p.scale);
             }
             fence_proxy_async_smem();
             named_bar_sync(2, 128);
-            if (threadIdx.x == 256) {
+            if (threadIdx.x == lead) {
               tma_reduce_add_4d(&p.tm_dq, sbase + C::OFF_DQS, box * 32, h, q0, I.b);
               bulk_commit_group();
             }
@@ -641,6 +671,10 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
             uint32_t v[32];
             tmem_ld32(tDQ + c * 32, v);
             tmem_wait_ld();
+            if (c + 1 == D / 32) {
+              tc_fence_before();
+              mbar_arrive(bar_dq_free(buf));
+            }
             if (q < p.Tq) {
 #pragma unroll
               for (int e = 0; e < 8; ++e)
@@ -649,19 +683,17 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_dkdv_kernel(const __grid_consta
                            __uint_as_float(v[4 * e + 3]) * p.scale);
             }
           }
-          tc_fence_before();
-          mbar_arrive(bar_dq_free(buf));
         }
       }
     }
     if constexpr (C::DQ_TMA) {
-      if (threadIdx.x == 256) bulk_wait_group0();
+      if (threadIdx.x == lead) bulk_wait_group0();
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 12) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -207,6 +207,17 @@ __device__ __forceinline__ void tmem_wait_st() {
 #define FA_W8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
                  "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : FA_R8(0)
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), FA_W8(0)
+               : "memory");
+}
+
 // 32 lanes x 32 bits, 16 consecutive columns: thread t of the warp gets
 // lane (addr.lane + t), columns addr.col .. addr.col+15.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {

@@ -139,6 +139,9 @@ static int device_setup() {
   return state[dev] - 1;
 }
 
+// Persistent decode grid: CTAs per SM.
+static constexpr int kDecodeCtasPerSm = 2;
+
 // Number of SMs of the current device (persistent grids use one CTA per SM).
 static int sm_count(int* n) {
   static int cache[kMaxDevices];
@@ -400,23 +403,27 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, c
   memset(&p, 0, sizeof(p));
   const size_t n = decode_nchunk(Tk_max, chunk);
   if (Tk_max > 0) {
-    st = make_tmap_4d(&p.tm_k, k_cache, d, Hkv, Tk_max, B, d, 64, false);
-    if (!st) st = make_tmap_4d(&p.tm_v, v_cache, d, Hkv, Tk_max, B, d, 64, false);
+    st = make_tmap_4d(&p.tm_k, k_cache, d, Hkv, Tk_max, B, 64, 64, true);
+    if (!st) st = make_tmap_4d(&p.tm_v, v_cache, d, Hkv, Tk_max, B, 64, 64, true);
     if (st) return st;
   }
+  if ((size_t)B * Hkv * n > (size_t)(1 << 30)) return FA_ERR_INVALID_ARG;
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.seqlens = seqlens_k;
   p.ws_o = reinterpret_cast<float*>(ws);
-  p.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) +
-                                      ((size_t)B * Hq * n * d * 4 + 255) / 256 * 256);
+  p.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + round256((size_t)B * Hq * n * d * 4));
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tk_max = Tk_max; p.chunk = chunk; p.nchunk = (int)n;
+  p.n_items = (int)((size_t)B * Hkv * n);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (Tk_max > 0) {
-    dim3 grid((unsigned)n, Hkv, B);
+    int nsm = 0;
+    if ((st = sm_count(&nsm))) return st;
+    // persistent: two CTAs per SM walk the (sequence, KV head, chunk) items
+    dim3 grid((unsigned)std::min<long long>(p.n_items, (long long)kDecodeCtasPerSm * nsm));
 #define FA_DEC_LAUNCH(DD, GG) \
     fa_decode_split_kernel<DD, GG><<<grid, DecCfg<DD, GG>::THREADS, DecCfg<DD, GG>::SMEM_BYTES, s>>>(p)
     if (d == 64) {
@@ -431,10 +438,16 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, c
   }
   const int warps = B * Hq;
   const int blocks = (warps * 32 + 255) / 256;
+  if (Tk_max > 0) {
+    if (d == 64)
+      fa_decode_combine_kernel<64><<<blocks, 256, 0, s>>>(p);
+    else
+      fa_decode_combine_kernel<128><<<blocks, 256, 0, s>>>(p);
+  }
   if (d == 64)
-    fa_decode_combine_kernel<64><<<blocks, 256, 0, s>>>(p);
+    fa_decode_empty_kernel<64><<<blocks, 256, 0, s>>>(p);
   else
-    fa_decode_combine_kernel<128><<<blocks, 256, 0, s>>>(p);
+    fa_decode_empty_kernel<128><<<blocks, 256, 0, s>>>(p);
   return launch_status();
 }
 

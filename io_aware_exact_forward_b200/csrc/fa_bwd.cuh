@@ -256,6 +256,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
   auto stg_par = [&](int g) { return (uint32_t)((g / C::NQ) & 1); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* stop_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
   float* dd_s = reinterpret_cast<float*>(smem + C::OFF_DD);
   auto aK = [&](int kvb) { return sbase + C::OFF_K + (2 * kvb) * C::TILE; };
@@ -268,6 +269,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    *stop_flag = 0;
     for (int s = 0; s < C::NQ; ++s) {
       mbar_init(bar_qdo_full(s), 1);
       mbar_init(bar_qdo_empty(s), 1);
@@ -633,15 +635,18 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         const int q0 = (I.qt_begin + it % I.nq) * 128;
         const uint32_t tDQ = tmem + C::TM_S0 + 128 * buf + lane_off;
         ok = __all_sync(0xffffffffu, mbar_wait(bar_dq_full(buf), (gi / C::NSBUF) & 1, wc));
-        if (!ok) break;
-        tc_fence_after();
         if constexpr (C::DQ_TMA) {
+          // The four warps meet at named barriers below: after an expired
+          // wait they still pass them, and all stop together at the end.
           uint32_t v[2][32];
-          tmem_ld32(tDQ, v[0]);
-          tmem_ld32(tDQ + 32, v[1]);
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(bar_dq_free(buf));
+          if (ok) {
+            tc_fence_after();
+            tmem_ld32(tDQ, v[0]);
+            tmem_ld32(tDQ + 32, v[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar_dq_free(buf));
+          }
           // fp32 staging, one 32-column box at a time (128-byte swizzle);
           // before each refill the previous bulk reduce must have read it.
 #pragma unroll
@@ -657,13 +662,20 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
                               __uint_as_float(v[box][4 * chunk + 3]) * p.scale);
             }
             fence_proxy_async_smem();
+            if (box == 1 && threadIdx.x == lead) *stop_flag = *abort_flag;
             named_bar_sync(2, 128);
-            if (threadIdx.x == lead) {
+            if (threadIdx.x == lead && !*stop_flag) {
               tma_reduce_add_4d(&p.tm_dq, sbase + C::OFF_DQS, box * 32, h, q0, I.b);
               bulk_commit_group();
             }
           }
+          if (*stop_flag) {
+            ok = false;
+            break;
+          }
         } else {
+          if (!ok) break;
+          tc_fence_after();
           const int q = q0 + r;
           float* dst = p.dq_acc + (((size_t)I.b * p.Tq + (q < p.Tq ? q : 0)) * p.Hq + h) * D;
 #pragma unroll

@@ -1,20 +1,31 @@
 // fa_decode.cuh -- split-KV decode: one query token per sequence against a
 // long KV cache.  The cache of every (sequence, KV head) is cut into chunks
-// that separate thread blocks process (FlashDecoding, "FlashAttention"
-// interview track, section "In practice"); each block writes its chunk's
+// that separate work items process (FlashDecoding, "FlashAttention"
+// interview track, section "In practice"); each item writes its chunk's
 // normalised output O_c and log-sum-exp LSE_c, and a second kernel merges
-// them: LSE = log sum_c e^{LSE_c}, O = sum_c e^{LSE_c - LSE} O_c -- the same
-// rescaling algebra as the online softmax of "Flash Attention: Why Memory
-// Traffic, Not Compute, Is the Bottleneck", section "Softmax Looks Like an
-// Obstacle".
+// them:
+//   LSE = log sum_c e^{LSE_c},  O = sum_c e^{LSE_c - LSE} O_c
+// -- the same rescaling algebra as the online softmax of "Flash Attention:
+// Why Memory Traffic, Not Compute, Is the Bottleneck", section "Softmax
+// Looks Like an Obstacle".
 //
 // Decode reads every cached key and value once and does ~4*G FLOPs per
 // cached bf16 element pair, so it is bound by HBM bandwidth ("Efficient
-// attention: memory-bound", the decoding paragraph).  The kernel therefore
-// uses CUDA cores (a GQA group has only G query rows, too few for a useful
-// tensor-core tile) and spends its effort on keeping loads in flight: a
-// producer warp streams 64-key K and V tiles with TMA into a ring of shared-
-// memory stages while four compute warps consume them.
+// attention: memory-bound", the decoding paragraph).  The kernel is built to
+// keep loads in flight and to spend little issue time per byte:
+//   * persistent CTAs (two per SM); a producer warp streams 64-key K and V
+//     tiles (K_0, V_0, K_1, V_1, ...) with TMA and the 128-byte swizzle into a
+//     ring of shared-memory stages, continuously across work items;
+//   * four compute warps, each owning 16 keys of every tile, run the dot
+//     products on the tensor cores with mma.sync (the G query rows of a GQA
+//     group padded to 16), keep an online softmax of their keys, and merge
+//     with the other warps by log-sum-exp at the end of the chunk.  A group
+//     has only G = 4 rows, far too few for a tcgen05 tile; mma.sync with
+//     padding costs a few instructions per 16 keys, so issue time stays far
+//     below the memory time.
+// Merging the chunks inside the split kernel (the last item of a sequence
+// to finish merging all of them) was measured 2.7x slower than the
+// separate merge kernel: the merging CTA stops streaming.
 #pragma once
 
 #include "fa_ptx.cuh"
@@ -22,7 +33,7 @@
 namespace fa {
 
 struct DecodeParams {
-  CUtensorMap tm_k;          // cache [B][Tk_max][Hkv][d], box {d, 1, 64, 1}, no swizzle
+  CUtensorMap tm_k;          // cache [B][Tk_max][Hkv][d], box {64, 1, 64, 1}, 128-byte swizzle
   CUtensorMap tm_v;
   const __nv_bfloat16* q;    // [B][Hq][d]
   const int* seqlens;        // [B]
@@ -31,6 +42,7 @@ struct DecodeParams {
   __nv_bfloat16* o;          // [B][Hq][d]
   float* lse;                // [B][Hq]
   int B, Hq, Hkv, Tk_max, chunk, nchunk;
+  int n_items;               // B * Hkv * nchunk (items past a sequence's end are skipped)
   float scale_log2;
   unsigned long long wait_limit_ns;
 };
@@ -38,230 +50,298 @@ struct DecodeParams {
 template <int D, int G>
 struct DecCfg {
   static constexpr int SUB = 64;                   // keys per TMA tile
-  static constexpr int STAGE_BYTES = SUB * D * 2;
-  static constexpr int NSTAGE = (D == 128) ? 4 : 8;
-  static constexpr int LPK = D / 8;                // lanes per key row (16 bytes each)
-  static constexpr int KPS = 32 / LPK;             // keys per warp step
-  static constexpr int NWARP = 4;                  // compute warps
+  static constexpr int NBOX = D / 64;              // 64-column swizzle boxes per tile
+  static constexpr int BOX_BYTES = SUB * 128;
+  static constexpr int STAGE_BYTES = NBOX * BOX_BYTES;
+  static constexpr int NSTAGE = (D == 128) ? (G >= 8 ? 5 : 6) : 10;  // two CTAs per SM
+  static constexpr int NWARP = 4;                  // compute warps, 16 keys of each tile each
   static constexpr int THREADS = (NWARP + 1) * 32;
-  static constexpr int MAX_CHUNK = 4096 / G;       // scores buffer: G * chunk floats
+  static constexpr int SEQ_CACHE = 1024;           // seqlens cached in shared memory
+  static constexpr int Q_BYTES = G * D * 2;
+  static constexpr int Q_STRIDE = (Q_BYTES + 127) / 128 * 128;
   static constexpr int OFF_RING = 0;
-  static constexpr int OFF_SCORE = NSTAGE * STAGE_BYTES;
-  static constexpr int OFF_RED = OFF_SCORE + G * MAX_CHUNK * 4;      // [NWARP][G][D] fp32
-  static constexpr int OFF_STAT = OFF_RED + NWARP * G * D * 4;       // m[G], l[G]
-  static constexpr int OFF_BAR = OFF_STAT + 2 * G * 4;
-  static constexpr int OFF_FLAG = OFF_BAR + 2 * NSTAGE * 8;
-  static constexpr int SMEM_BYTES = OFF_FLAG + 16 + 128;
+  static constexpr int OFF_Q = NSTAGE * STAGE_BYTES;                 // 2 stages
+  static constexpr int OFF_SEQ = OFF_Q + 2 * Q_STRIDE;
+  static constexpr int OFF_MRG = OFF_SEQ + SEQ_CACHE * 4;            // [NWARP][G][D] fp32
+  static constexpr int OFF_ML = OFF_MRG + NWARP * G * D * 4;         // m, l: [NWARP][G] each
+  static constexpr int OFF_BAR = OFF_ML + 2 * NWARP * G * 4;
+  static constexpr int NBAR = 2 * NSTAGE + 4;
+  static constexpr int OFF_FLAG = OFF_BAR + NBAR * 8;                // abort, stop flags
+  static constexpr int SMEM_BYTES = OFF_FLAG + 16 + 1024;            // + alignment slack
+  static constexpr float RESCALE_THRESHOLD = 8.0f;
 };
 
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.x4.m8n8.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.x4.trans.m8n8.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D(16x8 fp32) += A(16x16 bf16) * B(16x8 bf16)
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk `ch` (0 .. D/8-1) of row `key` in a stage made
+// of 64-column boxes with the 128-byte swizzle (chunk ^ row % 8).
+__device__ __forceinline__ uint32_t swz_off(int key, int ch) {
+  return (uint32_t)((ch >> 3) * 64 * 128 + key * 128 + (((ch & 7) ^ (key & 7)) << 4));
+}
+
+// Item k covers chunk k % nchunk of (sequence, KV head) k / nchunk.
 template <int D, int G>
 __global__ void __launch_bounds__(DecCfg<D, G>::THREADS)
 fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
   using C = DecCfg<D, G>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float* score = reinterpret_cast<float*>(smem + C::OFF_SCORE);
-  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
-  float* stat = reinterpret_cast<float*>(smem + C::OFF_STAT);
+  int* seq_s = reinterpret_cast<int*>(smem + C::OFF_SEQ);
+  float* mrg = reinterpret_cast<float*>(smem + C::OFF_MRG);
+  float* m_s = reinterpret_cast<float*>(smem + C::OFF_ML);
+  float* l_s = m_s + C::NWARP * G;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
+  volatile int* stop_flag = abort_flag + 1;
   auto bar_full = [&](int s) { return sbase + C::OFF_BAR + 8u * s; };
   auto bar_empty = [&](int s) { return sbase + C::OFF_BAR + 8u * (C::NSTAGE + s); };
-
-  const int c = blockIdx.x;        // chunk index
-  const int hkv = blockIdx.y;
-  const int b = blockIdx.z;
-  const int seqlen = p.seqlens[b];
-  const int k0 = c * p.chunk;
-  if (k0 >= seqlen) return;        // chunk past this sequence's end: nothing to do
-  const int nkeys = min(p.chunk, seqlen - k0);
-  const int nsub = (nkeys + C::SUB - 1) / C::SUB;
+  auto bar_qfull = [&](int s) { return sbase + C::OFF_BAR + 8u * (2 * C::NSTAGE + s); };
+  auto bar_qempty = [&](int s) { return sbase + C::OFF_BAR + 8u * (2 * C::NSTAGE + 2 + s); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   WaitCtl wc{abort_flag, p.wait_limit_ns};
 
+  for (int i = threadIdx.x; i < min(p.B, C::SEQ_CACHE); i += blockDim.x) seq_s[i] = p.seqlens[i];
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    *stop_flag = 0;
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(bar_full(s), 1);
       mbar_init(bar_empty(s), C::NWARP);
     }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_qfull(s), 1);
+      mbar_init(bar_qempty(s), C::NWARP);
+    }
     fence_barrier_init();
   }
   __syncthreads();
+  auto seqlen_of = [&](int b) { return b < C::SEQ_CACHE ? seq_s[b] : p.seqlens[b]; };
 
   if (warp == C::NWARP) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
       bool ok = true;
-      int issued = 0;
-      for (int t = 0; t < 2 * nsub && ok; ++t) {
-        const int s = t % C::NSTAGE;
-        const int round = t / C::NSTAGE;
-        if (round > 0) ok = mbar_wait(bar_empty(s), (round - 1) & 1, wc);
+      int t = 0, qi = 0;  // ring slot counter and item counter, continuous across items
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const int c = item % p.nchunk;
+        const int bh = item / p.nchunk;
+        const int b = bh / p.Hkv, hkv = bh % p.Hkv;
+        const int k0 = c * p.chunk;
+        const int seqlen = seqlen_of(b);
+        if (k0 >= seqlen) continue;
+        const int nsub = (min(p.chunk, seqlen - k0) + C::SUB - 1) / C::SUB;
+        // the G query rows of the group are contiguous: one bulk copy
+        const int qs = qi & 1;
+        if (qi >= 2) ok = mbar_wait(bar_qempty(qs), ((qi >> 1) - 1) & 1, wc);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar_full(s), C::STAGE_BYTES);
-        const int sub = t < nsub ? t : t - nsub;
-        tma_load_4d(sbase + C::OFF_RING + s * C::STAGE_BYTES, t < nsub ? &p.tm_k : &p.tm_v,
-                    bar_full(s), 0, hkv, k0 + sub * C::SUB, b);
-        ++issued;
+        mbar_arrive_expect_tx(bar_qfull(qs), C::Q_BYTES);
+        bulk_load(sbase + C::OFF_Q + qs * C::Q_STRIDE, p.q + ((size_t)b * p.Hq + hkv * G) * D, C::Q_BYTES,
+                  bar_qfull(qs));
+        ++qi;
+        // K_0, V_0, K_1, V_1, ... -- the order the compute warps consume
+        for (int i = 0; i < 2 * nsub && ok; ++i, ++t) {
+          const int s = t % C::NSTAGE;
+          const int round = t / C::NSTAGE;
+          if (round > 0) ok = mbar_wait(bar_empty(s), (round - 1) & 1, wc);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar_full(s), C::STAGE_BYTES);
+          for (int kb = 0; kb < C::NBOX; ++kb)
+            tma_load_4d(sbase + C::OFF_RING + s * C::STAGE_BYTES + kb * C::BOX_BYTES, (i & 1) ? &p.tm_v : &p.tm_k,
+                        bar_full(s), kb * 64, hkv, k0 + (i >> 1) * C::SUB, b);
+        }
       }
-      if (!ok)
-        for (int t = max(0, issued - C::NSTAGE); t < issued; ++t)
-          mbar_wait_drain(bar_full(t % C::NSTAGE), (t / C::NSTAGE) & 1, p.wait_limit_ns);
+      if (!ok) {
+        for (int k = max(0, t - C::NSTAGE); k < t; ++k)
+          mbar_wait_drain(bar_full(k % C::NSTAGE), (k / C::NSTAGE) & 1, p.wait_limit_ns);
+        for (int k = max(0, qi - 2); k < qi; ++k) mbar_wait_drain(bar_qfull(k & 1), (k >> 1) & 1, p.wait_limit_ns);
+      }
     }
     // the producer warp takes part in no named barrier below
     return;
   }
 
   // ------------------------------------------------------------ compute
-  const int kl = lane / C::LPK;            // key slot within a warp step
-  const int dl = (lane % C::LPK) * 8;      // first of this lane's 8 d-elements
-  float qf[G][8];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + hkv * G + g) * D + dl);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(h2[e]);
-      qf[g][2 * e] = f.x * p.scale_log2;
-      qf[g][2 * e + 1] = f.y * p.scale_log2;
-    }
-  }
-
+  // mma.sync fragment coordinates: row g = lane / 4 (query head of the group
+  // when g < G; rows G..15 are padding), column pair 2t, 2t+1 with t = lane % 4.
+  const int g = lane >> 2, t4 = lane & 3;
+  const bool real_row = g < G;
+  const int kw = warp * 16;                // this warp's 16 keys of every tile
   bool ok = true;
-  // Phase 1: scores (log2 units) for every key of the chunk.
-  for (int t = 0; t < nsub; ++t) {
-    const int s = t % C::NSTAGE;
-    ok = __all_sync(0xffffffffu, mbar_wait(bar_full(s), (t / C::NSTAGE) & 1, wc));
-    if (!ok) break;
-    const uint8_t* stage = smem + C::OFF_RING + s * C::STAGE_BYTES;
+  int t = 0, qi = 0;
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+    const int c = item % p.nchunk;
+    const int bh = item / p.nchunk;
+    const int b = bh / p.Hkv, hkv = bh % p.Hkv;
+    const int k0 = c * p.chunk;
+    const int seqlen = seqlen_of(b);
+    if (k0 >= seqlen) continue;
+    const int nkeys = min(p.chunk, seqlen - k0);
+    const int nsub = (nkeys + C::SUB - 1) / C::SUB;
+
+    // Q as the A operand (rows >= G are zero); scaling is applied to the
+    // fp32 scores, so the bf16 inputs enter the MMA unrounded.
+    uint32_t qa[D / 16][2];
+    {
+      const int qs = qi & 1;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_qfull(qs), (qi >> 1) & 1, wc));
+      const uint32_t* qrow =
+          reinterpret_cast<const uint32_t*>(smem + C::OFF_Q + qs * C::Q_STRIDE + (real_row ? g : 0) * D * 2);
 #pragma unroll
-    for (int st = 0; st < 16 / C::KPS; ++st) {
-      const int kk = warp * 16 + st * C::KPS + kl;   // key within the 64-key tile
-      const uint4 raw = *reinterpret_cast<const uint4*>(stage + kk * D * 2 + dl * 2);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      float kf[8];
+      for (int ks = 0; ks < D / 16; ++ks) {
+        qa[ks][0] = real_row ? qrow[ks * 8 + t4] : 0u;       // cols 16ks + 2t, +1
+        qa[ks][1] = real_row ? qrow[ks * 8 + 4 + t4] : 0u;   // cols 16ks + 8 + 2t, +1
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_qempty(qs));
+      ++qi;
+    }
+
+    // Online softmax over this warp's keys of the chunk (log2 units).
+    float m_run = -INFINITY, l_part = 0.f;
+    float oacc[D / 8][4];
+#pragma unroll
+    for (int nb = 0; nb < D / 8; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) oacc[nb][e] = 0.f;
+
+    for (int i = 0; i < nsub; ++i) {
+      // ---- K tile: scores of keys kw .. kw+15 of this 64-key tile
+      const int sK = t % C::NSTAGE;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_full(sK), (t / C::NSTAGE) & 1, wc));
+      ++t;
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (ok) {
+        const uint32_t st = sbase + C::OFF_RING + sK * C::STAGE_BYTES;
+        // matrices: (keys +0..7, cols +0..7), (+0..7, +8..15), (+8..15, +0..7), (+8..15, +8..15)
+        const int mrow = kw + ((lane >> 4) << 3) + (lane & 7);
+        const int mcol = (lane >> 3) & 1;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(st + swz_off(mrow, 2 * ks + mcol), b0, b1, b2, b3);
+          mma_16816(s0, qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+          mma_16816(s1, qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty(sK));
+      // this lane's keys: kw + 2t, +1 (s0) and kw + 8 + 2t, +1 (s1)
+      const int kb0 = i * C::SUB + kw + 2 * t4;
+      float sc[4] = {s0[0], s0[1], s1[0], s1[1]};
+      const int kk[4] = {kb0, kb0 + 1, kb0 + 8, kb0 + 9};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[e] = (kk[e] < nkeys && real_row) ? sc[e] * p.scale_log2 : -INFINITY;
+      float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      // Lazy rescale: move the reference only when the maximum grew by more
+      // than the threshold; l and O always share the reference.
+      if (mx > m_run + C::RESCALE_THRESHOLD || (m_run == -INFINITY && mx != -INFINITY)) {
+        const float alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mx);
+        l_part *= alpha;
+#pragma unroll
+        for (int nb = 0; nb < D / 8; ++nb) {
+          oacc[nb][0] *= alpha;
+          oacc[nb][1] *= alpha;
+        }
+        m_run = mx;
+      }
+      const float ref = (m_run == -INFINITY) ? 0.f : m_run;
+      float pv[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
-        kf[2 * e] = f.x;
-        kf[2 * e + 1] = f.y;
+        pv[e] = ex2_approx(sc[e] - ref);
+        l_part += pv[e];
       }
-      float acc[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaf(qf[g][e], kf[e], a);
-        acc[g] = a;
-      }
-#pragma unroll
-      for (int off = C::LPK / 2; off > 0; off >>= 1)
-#pragma unroll
-        for (int g = 0; g < G; ++g) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
-      const int key = t * C::SUB + kk;               // key within the chunk
-      if ((lane % C::LPK) == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) score[g * C::MAX_CHUNK + key] = key < nkeys ? acc[g] : -INFINITY;
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_empty(s));
-  }
-  named_bar_sync(1, C::NWARP * 32);
+      const uint32_t pa0 = pack_bf16x2(pv[0], pv[1]);   // row g, keys kw + 2t, +1
+      const uint32_t pa2 = pack_bf16x2(pv[2], pv[3]);   // row g, keys kw + 8 + 2t, +1
 
-  // Phase 2: softmax statistics per query head of the group; p = 2^{s - m}.
-  if (ok) {
-    for (int g = warp; g < G; g += C::NWARP) {
-      float mx = -INFINITY;
-      for (int k = lane; k < nkeys; k += 32) mx = fmaxf(mx, score[g * C::MAX_CHUNK + k]);
+      // ---- V tile: O += P V over the same 16 keys
+      const int sV = t % C::NSTAGE;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_full(sV), (t / C::NSTAGE) & 1, wc));
+      ++t;
+      if (ok) {
+        const uint32_t st = sbase + C::OFF_RING + sV * C::STAGE_BYTES;
+        // transposed matrices: (keys +0..7, d 8nb..), (keys +8..15, d 8nb..),
+        // (keys +0..7, d 8nb+8..), (keys +8..15, d 8nb+8..)
+        const int vrow = kw + ((lane >> 3) & 1) * 8 + (lane & 7);
+        const int vcol = lane >> 4;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      float sum = 0.f;
-      for (int k = lane; k < nsub * C::SUB; k += 32) {
-        const float e = k < nkeys ? ex2_approx(score[g * C::MAX_CHUNK + k] - mx) : 0.f;
-        score[g * C::MAX_CHUNK + k] = e;
-        sum += e;
+        for (int nb = 0; nb < D / 8; nb += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(st + swz_off(vrow, nb + vcol), b0, b1, b2, b3);
+          mma_16816(oacc[nb], pa0, 0u, pa2, 0u, b0, b1);
+          mma_16816(oacc[nb + 1], pa0, 0u, pa2, 0u, b2, b3);
+        }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      if (lane == 0) {
-        stat[g] = mx;
-        stat[G + g] = sum;
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty(sV));
     }
-  }
-  named_bar_sync(1, C::NWARP * 32);
 
-  // Phase 3: O_c = sum_k p_k V_k over the chunk's V tiles.
-  float acc[G][8];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-  for (int t = nsub; t < 2 * nsub && ok; ++t) {
-    const int s = t % C::NSTAGE;
-    ok = __all_sync(0xffffffffu, mbar_wait(bar_full(s), (t / C::NSTAGE) & 1, wc));
-    if (!ok) break;
-    const uint8_t* stage = smem + C::OFF_RING + s * C::STAGE_BYTES;
-#pragma unroll
-    for (int st = 0; st < 16 / C::KPS; ++st) {
-      const int kk = warp * 16 + st * C::KPS + kl;
-      const int key = (t - nsub) * C::SUB + kk;
-      const uint4 raw = *reinterpret_cast<const uint4*>(stage + kk * D * 2 + dl * 2);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      float vf[8];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
-        vf[2 * e] = f.x;
-        vf[2 * e + 1] = f.y;
+    // ---- merge the four warps by log-sum-exp
+    float l_row = l_part + __shfl_xor_sync(0xffffffffu, l_part, 1);
+    l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
+    if (real_row) {
+      if (t4 == 0) {
+        m_s[warp * G + g] = m_run;
+        l_s[warp * G + g] = l_row;
       }
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float pg = score[g * C::MAX_CHUNK + key];   // 0 for keys past the end
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg, vf[e], acc[g][e]);
-      }
+      for (int nb = 0; nb < D / 8; ++nb)
+        *reinterpret_cast<float2*>(&mrg[(warp * G + g) * D + nb * 8 + 2 * t4]) =
+            make_float2(oacc[nb][0], oacc[nb][1]);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_empty(s));
-  }
-  // Sum the key slots of the warp, then the warps, through shared memory.
+    named_bar_sync(1, C::NWARP * 32);
+    for (int idx = threadIdx.x; idx < G * D; idx += C::NWARP * 32) {
+      const int gg = idx / D, dd = idx % D;
+      float M = -INFINITY;
 #pragma unroll
-  for (int off = 16; off >= C::LPK; off >>= 1)
+      for (int w = 0; w < C::NWARP; ++w) M = fmaxf(M, m_s[w * G + gg]);
+      float L = 0.f, O = 0.f;
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], off);
-  if (lane < C::LPK) {
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red[(warp * G + g) * D + dl + e] = acc[g][e];
-  }
-  named_bar_sync(1, C::NWARP * 32);
-  if (!ok) return;
-  for (int i = threadIdx.x; i < G * D; i += C::NWARP * 32) {
-    const int g = i / D, dd = i % D;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < C::NWARP; ++w) v += red[(w * G + g) * D + dd];
-    const int h = hkv * G + g;
-    p.ws_o[(((size_t)b * p.Hq + h) * p.nchunk + c) * D + dd] = v / stat[G + g];
-  }
-  if (threadIdx.x < G) {
-    const int g = threadIdx.x;
-    const int h = hkv * G + g;
-    // natural-log LSE of the chunk: (m + log2 l) * ln 2
-    p.ws_lse[((size_t)b * p.Hq + h) * p.nchunk + c] = (stat[g] + log2f(stat[G + g])) * 0.69314718055994531f;
+      for (int w = 0; w < C::NWARP; ++w) {
+        const float mw = m_s[w * G + gg];
+        const float f = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+        L = fmaf(f, l_s[w * G + gg], L);
+        O = fmaf(f, mrg[(w * G + gg) * D + dd], O);
+      }
+      const size_t row = (size_t)b * p.Hq + hkv * G + gg;
+      p.ws_o[(row * p.nchunk + c) * D + dd] = O / L;
+      if (dd == 0) p.ws_lse[row * p.nchunk + c] = (M + log2f(L)) * 0.69314718055994531f;
+    }
+    // The merge scratch is reused by the next item only after this barrier.
+    // After an expired wait every compute warp has still passed the same
+    // named barriers; thread 0 samples the abort flag before the barrier so
+    // that all of them stop here together.
+    if (threadIdx.x == 0) *stop_flag = *abort_flag;
+    named_bar_sync(1, C::NWARP * 32);
+    if (*stop_flag) break;
   }
 }
 
-// One warp per (sequence, query head): merge the chunk partials by LSE.
+// Separate merge of the chunk partials: one warp per (sequence, query head).
 template <int D>
 __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const __grid_constant__ DecodeParams p) {
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -270,45 +350,63 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const __grid_con
   const int b = gw / p.Hq;
   const int seqlen = p.seqlens[b];
   const int nch = (seqlen + p.chunk - 1) / p.chunk;
+  if (nch == 0) return;  // written by fa_decode_empty_kernel
+  constexpr int E = D / 32;
   const float* lse_c = p.ws_lse + (size_t)gw * p.nchunk;
   const float* o_c = p.ws_o + (size_t)gw * p.nchunk * D;
-  constexpr int E = D / 32;  // elements per lane
+  float mx = -INFINITY;
+  for (int cc = lane; cc < nch; cc += 32) mx = fmaxf(mx, lse_c[cc]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float sum = 0.f;
+  for (int cc = lane; cc < nch; cc += 32) sum += ex2_approx((lse_c[cc] - mx) * 1.4426950408889634f);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  const float lse = mx + logf(sum);
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  if (nch == 0) {
-    if (lane == 0) p.lse[gw] = -INFINITY;
-  } else {
-    float mx = -INFINITY;
-    for (int c = lane; c < nch; c += 32) mx = fmaxf(mx, lse_c[c]);
+  int cc = 0;
+  for (; cc + 4 <= nch; cc += 4) {
+    float wgt[4], vals[4][E];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float sum = 0.f;
-    for (int c = lane; c < nch; c += 32) sum += ex2_approx((lse_c[c] - mx) * 1.4426950408889634f);
+    for (int u = 0; u < 4; ++u) {
+      wgt[u] = lse_c[cc + u];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    const float lse = mx + logf(sum);
-    for (int c = 0; c < nch; ++c) {
-      const float wgt = ex2_approx((lse_c[c] - lse) * 1.4426950408889634f);
-      const float* src = o_c + (size_t)c * D + lane * E;
-      if constexpr (E == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(src);
-        acc[0] = fmaf(wgt, v.x, acc[0]);
-        acc[1] = fmaf(wgt, v.y, acc[1]);
-        acc[2] = fmaf(wgt, v.z, acc[2]);
-        acc[3] = fmaf(wgt, v.w, acc[3]);
-      } else {
-        const float2 v = *reinterpret_cast<const float2*>(src);
-        acc[0] = fmaf(wgt, v.x, acc[0]);
-        acc[1] = fmaf(wgt, v.y, acc[1]);
-      }
+      for (int e = 0; e < E; ++e) vals[u][e] = o_c[(size_t)(cc + u) * D + lane * E + e];
     }
-    if (lane == 0) p.lse[gw] = lse;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float w = ex2_approx((wgt[u] - lse) * 1.4426950408889634f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(w, vals[u][e], acc[e]);
+    }
   }
+  for (; cc < nch; ++cc) {
+    const float w = ex2_approx((lse_c[cc] - lse) * 1.4426950408889634f);
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = fmaf(w, o_c[(size_t)cc * D + lane * E + e], acc[e]);
+  }
+  if (lane == 0) p.lse[gw] = lse;
   __nv_bfloat16* dst = p.o + (size_t)gw * D + lane * E;
 #pragma unroll
-  for (int e = 0; e < E; e += 2)
-    *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
+  for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
+}
+
+// Sequences with no cached key (seqlen 0) get O = 0 and LSE = -inf; every
+// other (sequence, head) is written by the merge kernel.
+template <int D>
+__global__ void __launch_bounds__(256) fa_decode_empty_kernel(const __grid_constant__ DecodeParams p) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= p.B * p.Hq) return;
+  const int b = gw / p.Hq;
+  if (p.seqlens[b] > 0) return;
+  constexpr int E = D / 32;
+  __nv_bfloat16* dst = p.o + (size_t)gw * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = 0u;
+  if (lane == 0) p.lse[gw] = -INFINITY;
 }
 
 }  // namespace fa

@@ -197,6 +197,16 @@ int fa_check(void* stream);
  */
 int fa_selftest_bounded_wait(int limit_us, void* stream);
 
+/*
+ * fa_selftest_exp2_poly -- evaluate, on n device floats x, the 2^x that the
+ * softmax kernels compute on the FMA pipe (Cody-Waite range reduction plus a
+ * degree-3 minimax polynomial), writing y.  Relative error below 1e-4 for x
+ * in [-125, 16]; x below -126 gives a non-negative value under 2^-125.
+ * Exposed so the approximation can be checked against a reference.  No
+ * counterpart on the pages: an implementation detail of the kernels.
+ */
+int fa_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -42,6 +42,7 @@ SIGNATURES = {
     "fa_decode_splitkv_noalloc": (_c_int, [_vp] * 6 + [_c_int] * 5 + [_c_float, _c_int, _vp]),
     "fa_check": (_c_int, [_vp]),
     "fa_selftest_bounded_wait": (_c_int, [_c_int, _vp]),
+    "fa_selftest_exp2_poly": (_c_int, [_vp, _vp, _c_int, _vp]),
 }
 
 

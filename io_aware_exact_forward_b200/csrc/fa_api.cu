@@ -483,6 +483,27 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
 }
 }  // namespace fa
 
+namespace fa {
+__global__ void selftest_exp2_poly_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 in = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  const float2 out = exp2_poly2(in);
+  y[i] = out.x;
+  if (i + 1 < n) y[i + 1] = out.y;
+}
+}  // namespace fa
+
+extern "C" int fa_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  int st = device_setup();
+  if (st) return st;
+  const int pairs = (n + 1) / 2;
+  selftest_exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return launch_status();
+}
+
 extern "C" int fa_selftest_bounded_wait(int limit_us, void* stream) {
   if (limit_us < 1 || limit_us > 1000000) return FA_ERR_INVALID_ARG;
   int st = device_setup();

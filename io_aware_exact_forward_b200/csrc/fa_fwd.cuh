@@ -72,6 +72,10 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
   static constexpr float RESCALE_THRESHOLD = 8.0f;
+  // Pairs of S columns whose exponentials use exp2_poly2 (3 of every 8 at
+  // d = 128, where the shared MUFU unit limits the softmax; none at d = 64,
+  // where the extra FMA-pipe instructions cost more than they save).
+  static constexpr bool poly_pair(int c) { return D == 128 && ((c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6); }
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
 };
 
@@ -320,10 +324,17 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
         const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nref = make_float2(-ref, -ref);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const bool masked = __any_sync(0xffffffffu, nvalid < C::BN);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(su[2 * c]), __uint_as_float(su[2 * c + 1])), sl2, nref);
-          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          // Part of the exponentials go to the FMA pipe so that the MUFU
+          // unit, shared by both softmax warpgroups, is not the bottleneck.
+          float2 pr = C::poly_pair(c) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          if (C::poly_pair(c) && masked) {
+            if (2 * c >= nvalid) pr.x = 0.f;
+            if (2 * c + 1 >= nvalid) pr.y = 0.f;
+          }
           acc[c & 3] = __fadd2_rn(acc[c & 3], pr);
           su[c] = pack_bf16x2(pr.x, pr.y);
         }

@@ -299,6 +299,31 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x for a pair of floats on the FMA pipe instead of the MUFU unit.
+// Cody-Waite range reduction: x = n + f with n = round(x) (from the bits of
+// x + 1.5*2^23) and f in [-1/2, 1/2]; 2^f by the degree-3 minimax polynomial
+// of fit_exp2_poly.py (Remez exchange on relative error, 7.5e-5 at most);
+// 2^n added into the exponent bits.  x is clamped below at -126 (a lower
+// clamp would wrap the exponent field of p < 1 into the sign bit), so inputs
+// under -126 (including -inf) give a denormal near 2^-126, not 0: callers
+// that need exact zeros (masked entries) must select them.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
+  const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                        make_float2(0.2426111251115799f, 0.2426111251115799f));
+  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  // the low mantissa bits of t hold n; shifting them to the exponent field
+  // multiplies by 2^n (the magic's own bits vanish in the shift)
+  return make_float2(__int_as_float(__float_as_int(p.x) + (int)((uint32_t)__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (int)((uint32_t)__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

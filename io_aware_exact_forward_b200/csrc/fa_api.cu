@@ -329,10 +329,15 @@ int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO
   p.n_kv_tiles = (Tk + 127) / 128;
   p.n_items = p.n_kv_tiles * B * Hkv;
   p.wait_limit_ns = kWaitLimitNs;
-  // One CTA per item (the kernel also runs persistently over a smaller grid;
-  // measured slower here because an item's K/V reload then waits on the
-  // previous item's last MMAs).
-  dim3 grid(p.n_items);
+  // Non-causal d = 64: one persistent CTA per SM, whose next item's K/V
+  // load overlaps the current item (two K/V buffers); items are all the
+  // same length there.  Otherwise one CTA per item: causal items differ in
+  // length and the hardware scheduler balances them, and at d = 128 there
+  // is room for one K/V buffer only.
+  int nsm = 0;
+  if ((st = sm_count(&nsm))) return st;
+  const bool persistent = d == 64 && !causal;
+  dim3 grid(persistent ? std::min(p.n_items, nsm) : p.n_items);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64)
     fa_bwd_dkdv_kernel<64><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);

@@ -21,13 +21,17 @@
 //                        shared memory as an A operand)
 //                  dK += dS^T Q                         (TS MMA)
 //                  dQ_tile = dS K                       (SS MMA)
-//                The next tile's dP^T MMA is issued as soon as the dS warps
-//                have read this tile's dP^T.
-//                dQ_tile is read by a second warpgroup and added into an fp32
-//                accumulator in global memory with vector reductions (every
-//                KV tile contributes to every query row it sees).  dK and dV
-//                are summed over the group's heads in tensor memory, so the
-//                GQA sum needs no atomics.
+//                At d = 64 (two S^T buffers) the next tile's S^T is issued
+//                ahead and its dP^T as soon as the dS warps have read this
+//                tile's; at d = 128 (one S^T buffer) dQ_tile lands in the dP^T
+//                columns, so that the next S^T follows dQ at once and the
+//                next dP^T follows the dQ read-out.
+//                dQ_tile is read by a second warpgroup, staged in shared
+//                memory and added into an fp32 accumulator in global memory
+//                with bulk tensor reduce-adds (every KV tile contributes to
+//                every query row it sees).  dK and dV are summed over the
+//                group's heads in tensor memory, so the GQA sum needs no
+//                atomics.
 //   dq_convert   dq = bf16(accumulator).
 // Warp roles in dkdv: 0-7 P^T and 8-15 dS (two warps per TMEM lane quarter,
 // one per half of the 128 query columns, so that one warp computes while the
@@ -133,12 +137,6 @@ struct BwdParams {
   unsigned long long wait_limit_ns;
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
-
 // Bulk tensor reduce-add of a shared-memory tile into global memory (fp32).
 __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* m, uint32_t src, int c0, int c1,
                                                   int c2, int c3) {
@@ -159,29 +157,35 @@ struct BwdCfg {
   static constexpr int NBOX = D / 64;
   static constexpr int BOX_BYTES = 128 * 128;
   static constexpr int TILE = NBOX * BOX_BYTES;         // 128 rows x D bf16
-  // d = 64: two S^T buffers in tensor memory, two K/V buffers in shared
-  // memory (the next item's K/V load overlaps this item) and dQ leaves
-  // through a shared-memory tile and a bulk tensor reduce.  d = 128: one of
-  // each (tensor and shared memory are full) and dQ leaves through vector
-  // reductions.
+  // d = 64: two S^T buffers in tensor memory, two K/V buffers and three
+  // Q/dO stages in shared memory (the next item's K/V load overlaps this
+  // item) and one 32-column fp32 box for staging dQ.  d = 128: one S^T
+  // buffer and one K/V buffer (tensor and shared memory are full), two Q
+  // stages but a single dO buffer with its own barriers (the next dO is
+  // loaded between this tile's dV and the next tile's dP^T), which leaves
+  // room for two dQ staging boxes.  The staged boxes go out with bulk
+  // tensor reduce-adds.
   static constexpr int NSBUF = (D == 64) ? 2 : 1;
   static constexpr int NKV = (D == 64) ? 2 : 1;
-  static constexpr bool DQ_TMA = (D == 64);
-  static constexpr int NQ = (D == 64) ? 3 : 2;          // Q / dO / LSE2 / D stages
+  static constexpr bool SPLIT_DO = (D == 128);
+  static constexpr int NQ = (D == 64) ? 3 : 2;          // Q / LSE2 / D (and dO) stages
+  static constexpr int NDO = SPLIT_DO ? 1 : NQ;         // dO buffers
+  static constexpr int NDQS = (D == 128) ? 2 : 1;       // dQ staging boxes
   static constexpr int OFF_K = 0;                       // NKV buffers of (K, V)
   static constexpr int OFF_Q = 2 * NKV * TILE;          // NQ stages
-  static constexpr int OFF_DO = OFF_Q + NQ * TILE;      // NQ stages
-  static constexpr int OFF_DS = OFF_DO + NQ * TILE;     // 128 x 128 bf16, 2 boxes
-  // fp32 staging of 32 dQ columns (one 128-byte swizzled box), reused for
-  // each box of the tile (DQ_TMA only)
+  static constexpr int OFF_DO = OFF_Q + NQ * TILE;      // NDO buffers
+  static constexpr int OFF_DS = OFF_DO + NDO * TILE;    // 128 x 128 bf16, 2 boxes
+  // fp32 staging of 32 dQ columns per box (128-byte swizzle), reused across
+  // the boxes of the tile
   static constexpr int OFF_DQS = OFF_DS + 2 * BOX_BYTES;
-  static constexpr int DQS_BYTES = DQ_TMA ? 128 * 32 * 4 : 0;
+  static constexpr int DQS_BYTES = NDQS * 128 * 32 * 4;
   static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;   // [NQ][128] f32
   static constexpr int OFF_DD = OFF_LSE + NQ * 128 * 4; // [NQ][128] f32
   static constexpr int OFF_BAR = OFF_DD + NQ * 128 * 4;
   // kv_full[2], kv_empty[2], qdo_full[3], qdo_empty[3], s_full[2], p_full[2],
-  // dp_full, ds_full, dq_full[2], dq_free[2], dkdv_done, mma_done, dp_free
-  static constexpr int NBAR = 23;
+  // dp_full, ds_full, dq_full[2], dq_free[2], dkdv_done, mma_done, dp_free,
+  // do_full, p_read, do_empty
+  static constexpr int NBAR = 26;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   // warps 0-7 P^T (two per TMEM lane quarter, one per half of the query
@@ -198,6 +202,8 @@ struct BwdCfg {
   static constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 1, 1);
   static_assert(TM_DP + 128 <= TMEM_COLS, "tensor memory overflow");
+  static_assert(OFF_DQS % 1024 == 0 && OFF_DS % 1024 == 0 && OFF_DO % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
   static_assert(NQ <= 3, "barrier slots");
 };
@@ -251,6 +257,9 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
   const uint32_t bar_dkdv_done = bar0 + 8u * 20;
   const uint32_t bar_mma_done = bar0 + 8u * 21;
   const uint32_t bar_dp_free = bar0 + 8u * 22;
+  const uint32_t bar_do_full = bar0 + 8u * 23;   // single dO buffer (d = 128)
+  const uint32_t bar_p_read = bar0 + 8u * 24;    // the dS warps hold this tile's P^T
+  const uint32_t bar_do_empty = bar0 + 8u * 25;
   // Q/dO stage of global iteration g and the parity of its use of that stage.
   auto stg = [&](int g) { return g % C::NQ; };
   auto stg_par = [&](int g) { return (uint32_t)((g / C::NQ) & 1); };
@@ -287,6 +296,9 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
     mbar_init(bar_ds_full, 256);
     mbar_init(bar_dkdv_done, 1);
     mbar_init(bar_mma_done, 1);
+    mbar_init(bar_do_full, 1);
+    mbar_init(bar_do_empty, 1);
+    mbar_init(bar_p_read, 256);
     fence_barrier_init();
   }
   if (warp == C::MMA_WARP) {
@@ -306,7 +318,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
       bool ok = true;
-      int gi = 0, ki = 0, issued_kv = 0;
+      int gi = 0, ki = 0, issued_kv = 0, n_do = 0;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const BwdItem I = bwd_item(p, item);
         if (I.n_it == 0) continue;
@@ -326,15 +338,25 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           if (gi >= C::NQ) ok = mbar_wait(bar_qdo_empty(s), stg_par(gi) ^ 1u, wc);
           if (!ok) break;
           const size_t rbase = ((size_t)I.b * p.Hq + h) * p.Tq_pad + q0;
-          mbar_arrive_expect_tx(bar_qdo_full(s), 2 * C::TILE + 2 * 512);
+          mbar_arrive_expect_tx(bar_qdo_full(s), (C::SPLIT_DO ? 1 : 2) * C::TILE + 2 * 512);
           for (int kb = 0; kb < C::NBOX; ++kb) {
             tma_load_4d(sbase + C::OFF_Q + s * C::TILE + kb * C::BOX_BYTES, &p.tm_q, bar_qdo_full(s), kb * 64, h,
                         q0, I.b);
-            tma_load_4d(sbase + C::OFF_DO + s * C::TILE + kb * C::BOX_BYTES, &p.tm_do, bar_qdo_full(s), kb * 64,
-                        h, q0, I.b);
+            if (!C::SPLIT_DO)
+              tma_load_4d(sbase + C::OFF_DO + s * C::TILE + kb * C::BOX_BYTES, &p.tm_do, bar_qdo_full(s),
+                          kb * 64, h, q0, I.b);
           }
           bulk_load(sbase + C::OFF_LSE + s * 512, p.lse2 + rbase, 512, bar_qdo_full(s));
           bulk_load(sbase + C::OFF_DD + s * 512, p.Dv + rbase, 512, bar_qdo_full(s));
+          if (C::SPLIT_DO) {
+            // the single dO buffer: free once the previous tile's dV is done
+            if (gi >= 1) ok = mbar_wait(bar_do_empty, (gi - 1) & 1, wc);
+            if (!ok) break;
+            mbar_arrive_expect_tx(bar_do_full, C::TILE);
+            for (int kb = 0; kb < C::NBOX; ++kb)
+              tma_load_4d(sbase + C::OFF_DO + kb * C::BOX_BYTES, &p.tm_do, bar_do_full, kb * 64, h, q0, I.b);
+            ++n_do;
+          }
         }
         ++ki;
       }
@@ -343,6 +365,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           mbar_wait_drain(bar_kv_full(k % C::NKV), (k / C::NKV) & 1, p.wait_limit_ns);
         for (int g = max(0, gi - C::NQ); g <= gi; ++g)
           mbar_wait_drain(bar_qdo_full(stg(g)), stg_par(g), p.wait_limit_ns);
+        if (n_do > 0) mbar_wait_drain(bar_do_full, (n_do - 1) & 1, p.wait_limit_ns);
       }
     }
   } else if (warp == C::MMA_WARP) {
@@ -352,7 +375,8 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
       auto tS = [&](int buf) { return tmem + C::TM_S0 + 128 * buf; };
       const uint32_t aDS = sbase + C::OFF_DS;
       auto aQ = [&](int g) { return sbase + C::OFF_Q + stg(g) * C::TILE; };
-      auto aDO = [&](int g) { return sbase + C::OFF_DO + stg(g) * C::TILE; };
+      auto aDO = [&](int g) { return sbase + C::OFF_DO + (C::SPLIT_DO ? 0 : stg(g) * C::TILE); };
+      auto wait_do = [&](int g) { return !C::SPLIT_DO || mbar_wait(bar_do_full, g & 1, wc); };
       auto kdesc = [&](uint32_t base, int k) {  // K-major tile, k-th 16-element slice of d
         return smem_desc_sw128(base + (k >> 2) * C::BOX_BYTES + (k & 3) * 32, 16, 1024);
       };
@@ -380,6 +404,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         if (!started) {
           ok = mbar_wait(bar_kv_full(kvb), (ki / C::NKV) & 1, wc);
           if (ok) ok = mbar_wait(bar_qdo_full(stg(0)), stg_par(0), wc);
+          if (ok) ok = wait_do(0);
           if (!ok) break;
           tc_fence_after();
           issue_s(0, kvb);
@@ -409,7 +434,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             issue_s(gi + 1, kvb_next);
           }
           // P^T of query half h sits in columns [64h, 64h+32) of the S^T
-          // buffer, dS^T of that half in [64h+32, 64h+64).
+          // buffer.
           auto p_col = [](int k) { return (k < 4) ? k * 8 : 64 + (k - 4) * 8; };
           ok = mbar_wait(bar_p_full(buf), (gi / C::NSBUF) & 1, wc);
           if (!ok) break;
@@ -417,34 +442,52 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mma_ts(tDV, tS(buf) + p_col(k), mndesc(aDO(gi), k), C::IDESC_TS, it > 0 || k > 0);
-          if (has_next) {
+          if (C::SPLIT_DO) mma_commit(bar_do_empty);
+          if (C::NSBUF == 2 && has_next) {
             // dP^T of the next tile as soon as the dS warps have read this one.
             ok = mbar_wait(bar_dp_free, gi & 1, wc);
-            if (ok && C::NSBUF == 1) ok = wait_next_operands();
             if (!ok) break;
             tc_fence_after();
             issue_dp(gi + 1, kvb_next);
           }
+          if (C::NSBUF == 1 && has_next) {
+            // With one S^T buffer the next S^T follows dV (queued behind it)
+            // once the dS warps hold this tile's P^T in registers.
+            ok = wait_next_operands();
+            if (ok) ok = mbar_wait(bar_p_read, gi & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(gi + 1, kvb_next);
+          }
           ok = mbar_wait(bar_ds_full, gi & 1, wc);
           if (!ok) break;
           tc_fence_after();
+          // dK += dS^T Q with dS^T read from the shared dS tile (key rows,
+          // query columns: K-major for this product).  Its completion frees
+          // the Q stage.
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_ts(tDK, tS(buf) + 32 + p_col(k), mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
+            mma_ss(tDK, kdesc(aDS, k), mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
           mma_commit(bar_qdo_empty(stg(gi)));
-          // dQ = dS K into this tile's S^T buffer (P^T and dS^T read above).
+          // dQ = dS K: with two S^T buffers into this tile's (P^T was read
+          // above); with one, into the dP^T columns, which the dS warps have
+          // read (the S^T buffer already holds the next S^T).  Its
+          // completion frees the dS tile.
+          const uint32_t tDQ = C::NSBUF == 1 ? tDP : tS(buf);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mma_ss(tS(buf), mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
+          for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
           mma_commit(bar_dq_full(buf));
           if (last) {
             mma_commit(bar_kv_empty(kvb));
             mma_commit(bar_dkdv_done);
           }
           if (C::NSBUF == 1 && has_next) {
+            // The next dP^T reuses the dQ columns: after the dQ read-out.
             ok = mbar_wait(bar_dq_free(0), gi & 1, wc);
+            if (ok) ok = wait_do(gi + 1);
             if (!ok) break;
             tc_fence_after();
-            issue_s(gi + 1, kvb_next);
+            issue_dp(gi + 1, kvb_next);
           }
         }
         ++ki;
@@ -562,44 +605,46 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
       const BwdItem I = bwd_item(p, item);
       for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
         const int s = stg(gi), buf = gi % C::NSBUF;
-        const uint32_t tP = tmem + C::TM_S0 + 128 * buf + lane_off + 64 * half;  // P^T, then dS^T at +32
+        const uint32_t tP = tmem + C::TM_S0 + 128 * buf + lane_off + 64 * half;  // P^T (bf16 pairs)
         ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), stg_par(gi), wc));
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_p_full(buf), (gi / C::NSBUF) & 1, wc));
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, gi & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+        // P^T of this warp's 64 query columns into registers at once, so
+        // that the S^T buffer can take the next S^T.
+        uint32_t pp[32];
+        tmem_ld32(tP, pp);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_p_read);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, gi & 1, wc));
         if (!ok) break;
         tc_fence_after();
         const float* drow = dd_s + s * 128 + 64 * half;
-        uint32_t pp[2][8], dp[2][16];
-        tmem_ld8(tP, pp[0]);
-        tmem_ld16(tDP, dp[0]);
+        // Four chunks of 16 query columns; dS overwrites P in pp.
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          uint32_t dp[16];
+          tmem_ld16(tDP + 16 * c, dp);
           tmem_wait_ld();
-          if (c + 1 < 4) {
-            tmem_ld8(tP + (c + 1) * 8, pp[(c + 1) & 1]);
-            tmem_ld16(tDP + (c + 1) * 16, dp[(c + 1) & 1]);
-          } else {
+          if (c == 3) {
             // every dP^T column of this warp has been read
             tc_fence_before();
             mbar_arrive(bar_dp_free);
           }
-          const uint32_t* cp = pp[c & 1];
-          const uint32_t* cd = dp[c & 1];
-          uint32_t ds[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cp[e]));
-            const float2 dd = *reinterpret_cast<const float2*>(drow + c * 16 + 2 * e);
-            const float2 t = __fadd2_rn(make_float2(__uint_as_float(cd[2 * e]), __uint_as_float(cd[2 * e + 1])),
+            const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[8 * c + e]));
+            const float2 dd = *reinterpret_cast<const float2*>(drow + 16 * c + 2 * e);
+            const float2 t = __fadd2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
                                         make_float2(-dd.x, -dd.y));
             const float2 r = __fmul2_rn(pf, t);
-            ds[e] = pack_bf16x2(r.x, r.y);
+            pp[8 * c + e] = pack_bf16x2(r.x, r.y);
           }
-          tmem_st8(tP + 32 + c * 8, ds);
           if (c == 0 && gi > 0) {
-            // The shared dS tile is still the A operand of the previous
-            // tile's dQ MMA until that MMA completes (this tile's dP^T can
-            // complete before it).
+            // The shared dS tile is still an operand of the previous tile's
+            // dK and dQ MMAs until they complete (this tile's dP^T can
+            // complete before them).
             ok = __all_sync(0xffffffffu,
                             mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
             if (!ok) break;
@@ -607,14 +652,13 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           // dS into shared memory: row j of box `half`, 16-byte chunks 2c and
           // 2c+1, 128-byte swizzle (chunk ^ (row % 8)).
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int chunk = 2 * c + cc;
+          for (int q = 0; q < 2; ++q) {
+            const int chunk = 2 * c + q;
             *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (j & 7)) << 4)) =
-                make_uint4(ds[4 * cc], ds[4 * cc + 1], ds[4 * cc + 2], ds[4 * cc + 3]);
+                make_uint4(pp[8 * c + 4 * q], pp[8 * c + 4 * q + 1], pp[8 * c + 4 * q + 2], pp[8 * c + 4 * q + 3]);
           }
         }
         if (!ok) break;
-        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar_ds_full);
@@ -633,74 +677,61 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         const int buf = gi % C::NSBUF;
         const int h = I.hkv * G + it / I.nq;
         const int q0 = (I.qt_begin + it % I.nq) * 128;
-        const uint32_t tDQ = tmem + C::TM_S0 + 128 * buf + lane_off;
+        const uint32_t tDQ = tmem + (C::NSBUF == 1 ? C::TM_DP : C::TM_S0 + 128 * buf) + lane_off;
         ok = __all_sync(0xffffffffu, mbar_wait(bar_dq_full(buf), (gi / C::NSBUF) & 1, wc));
-        if constexpr (C::DQ_TMA) {
-          // The four warps meet at named barriers below: after an expired
-          // wait they still pass them, and all stop together at the end.
+        // The four warps meet at named barriers below: after an expired wait
+        // they still pass them, and all stop together at the end.
+        if (ok) tc_fence_after();
+#pragma unroll
+        for (int pr = 0; pr < D / 64; ++pr) {
+          // 64 columns (two fp32 boxes) per pass; the tensor-memory columns
+          // are released after the last pass's loads.
           uint32_t v[2][32];
           if (ok) {
-            tc_fence_after();
-            tmem_ld32(tDQ, v[0]);
-            tmem_ld32(tDQ + 32, v[1]);
+            tmem_ld32(tDQ + 64 * pr, v[0]);
+            tmem_ld32(tDQ + 64 * pr + 32, v[1]);
             tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar_dq_free(buf));
+            if (pr + 1 == D / 64) {
+              tc_fence_before();
+              mbar_arrive(bar_dq_free(buf));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[0][i] = v[1][i] = 0u;  // a stopped warp adds nothing
           }
-          // fp32 staging, one 32-column box at a time (128-byte swizzle);
-          // before each refill the previous bulk reduce must have read it.
 #pragma unroll
           for (int box = 0; box < 2; ++box) {
-            if (threadIdx.x == lead) bulk_wait_group_read0();
-            named_bar_sync(2, 128);
+            // Before a staging box is refilled, the bulk reduce that last
+            // read it must have finished reading.
+            const uint32_t slot = C::OFF_DQS + (box % C::NDQS) * C::BOX_BYTES;
+            if (box == 0 || C::NDQS == 1) {
+              if (threadIdx.x == lead) bulk_wait_group_read0();
+              named_bar_sync(2, 128);
+            }
 #pragma unroll
             for (int chunk = 0; chunk < 8; ++chunk) {
-              *reinterpret_cast<float4*>(smem + C::OFF_DQS + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+              *reinterpret_cast<float4*>(smem + slot + r * 128 + ((chunk ^ (r & 7)) << 4)) =
                   make_float4(__uint_as_float(v[box][4 * chunk]) * p.scale,
                               __uint_as_float(v[box][4 * chunk + 1]) * p.scale,
                               __uint_as_float(v[box][4 * chunk + 2]) * p.scale,
                               __uint_as_float(v[box][4 * chunk + 3]) * p.scale);
             }
             fence_proxy_async_smem();
-            if (box == 1 && threadIdx.x == lead) *stop_flag = *abort_flag;
+            if (pr + 1 == D / 64 && box == 1 && threadIdx.x == lead) *stop_flag = *abort_flag;
             named_bar_sync(2, 128);
             if (threadIdx.x == lead && !*stop_flag) {
-              tma_reduce_add_4d(&p.tm_dq, sbase + C::OFF_DQS, box * 32, h, q0, I.b);
+              tma_reduce_add_4d(&p.tm_dq, sbase + slot, (2 * pr + box) * 32, h, q0, I.b);
               bulk_commit_group();
             }
           }
-          if (*stop_flag) {
-            ok = false;
-            break;
-          }
-        } else {
-          if (!ok) break;
-          tc_fence_after();
-          const int q = q0 + r;
-          float* dst = p.dq_acc + (((size_t)I.b * p.Tq + (q < p.Tq ? q : 0)) * p.Hq + h) * D;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tDQ + c * 32, v);
-            tmem_wait_ld();
-            if (c + 1 == D / 32) {
-              tc_fence_before();
-              mbar_arrive(bar_dq_free(buf));
-            }
-            if (q < p.Tq) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
-                           __uint_as_float(v[4 * e + 1]) * p.scale, __uint_as_float(v[4 * e + 2]) * p.scale,
-                           __uint_as_float(v[4 * e + 3]) * p.scale);
-            }
-          }
+        }
+        if (*stop_flag) {
+          ok = false;
+          break;
         }
       }
     }
-    if constexpr (C::DQ_TMA) {
-      if (threadIdx.x == lead) bulk_wait_group0();
-    }
+    if (threadIdx.x == lead) bulk_wait_group0();
   }
 
   tc_fence_before();

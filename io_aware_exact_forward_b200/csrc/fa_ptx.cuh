@@ -51,6 +51,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// try_wait with the default suspend-time limit.  (A short explicit hint
+// halves the hand-off latency between two otherwise idle warps, but the
+// extra polling slowed the backward kernel, where most warps wait at once.)
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

@@ -36,7 +36,11 @@ Readings where the pages are silent (each is also listed in the design notes):
   LSE = -inf and zero gradients;
 * GQA maps query head h to KV head h // (Hq // Hkv) (contiguous groups);
 * D_i of the backward pass is sum_j P_ij dP_ij (the softmax Jacobian), not the
-  rowsum(dO*O) shortcut the kernels use.
+  rowsum(dO*O) shortcut the kernels use;
+* sliding window ([FA §"In practice"] names "sliding windows" next to GQA and
+  causal masks, without a definition): a causal local window of W >= 1 keys,
+  query i sees key j iff i + (Tk - Tq) - W < j <= i + (Tk - Tq), i.e. its own
+  diagonal key and the W - 1 keys before it.  W >= Tk is the causal mask.
 
 Layouts follow the library: q, o, dq are [B, Tq, Hq, d]; k, v, dk, dv are
 [B, Tk, Hkv, d]; lse is [B, Hq, Tq].  All arrays are float64.
@@ -50,6 +54,7 @@ import numpy as np
 
 __all__ = [
     "causal_visible",
+    "window_visible",
     "head_forward",
     "head_backward",
     "attention_forward",
@@ -71,6 +76,20 @@ def causal_visible(i: int, j, Tq: int, Tk: int):
     return j <= i + (Tk - Tq)
 
 
+def window_visible(i, j, Tq: int, Tk: int, window: int):
+    """Sliding-window rule (reading of [FA §"In practice"]): the causal rule
+    plus j > i + (Tk - Tq) - window, so each query sees its `window` most
+    recent keys, its diagonal key included."""
+    off = Tk - Tq
+    return (j <= i + off) & (j > i + off - window)
+
+
+def _visible(i, j, Tq: int, Tk: int, causal: bool, window):
+    if window is not None:
+        return window_visible(i, j, Tq, Tk, window)
+    return causal_visible(i, j, Tq, Tk)
+
+
 def _kv_head(h: int, Hq: int, Hkv: int) -> int:
     """GQA head map (reading of [FA §"In practice"]): contiguous groups."""
     return h // (Hq // Hkv)
@@ -84,14 +103,14 @@ def _visible_keys(r1: int, Tq: int, Tk: int, causal: bool) -> int:
     return max(0, min(Tk, (r1 - 1) + (Tk - Tq) + 1))
 
 
-def _masked_scores(qp, kh, r0, Tq, Tk, scale, causal):
+def _masked_scores(qp, kh, r0, Tq, Tk, scale, causal, window=None):
     """S = scale * Q K^T for query rows r0.. of the panel [EFF §"Standard
     attention, kernel by kernel", step 1], with masked entries set to -inf."""
     S = scale * (qp @ kh.T)
-    if causal:
+    if causal or window is not None:
         rows = np.arange(r0, r0 + qp.shape[0])[:, None]
         cols = np.arange(kh.shape[0])[None, :]
-        S = np.where(causal_visible(rows, cols, Tq, Tk), S, -np.inf)
+        S = np.where(_visible(rows, cols, Tq, Tk, causal, window), S, -np.inf)
     return S
 
 
@@ -111,13 +130,17 @@ def _softmax_stats(S):
     return lse, P
 
 
-def head_forward(qh, kh, vh, scale: float, causal: bool, rows=None):
+def head_forward(qh, kh, vh, scale: float, causal: bool, rows=None, window=None):
     """One head: O = softmax(scale * Q K^T [+ mask]) V and LSE per row.
 
     qh [Tq, d], kh/vh [Tk, d].  ``rows`` optionally restricts the output to a
     subset of query rows (each row is independent, so this is the same
-    definition evaluated only where asked).  Returns (O [n, d], LSE [n]).
+    definition evaluated only where asked).  ``window`` (an int >= 1, or
+    None) applies the sliding-window rule, which includes the causal one.
+    Returns (O [n, d], LSE [n]).
     """
+    if window is not None:
+        causal = True
     Tq, Tk = qh.shape[0], kh.shape[0]
     if rows is None:
         rows = np.arange(Tq)
@@ -129,18 +152,21 @@ def head_forward(qh, kh, vh, scale: float, causal: bool, rows=None):
         nk = _visible_keys(int(sel.max()) + 1, Tq, Tk, causal) if len(sel) else 0
         S = scale * (qh[sel] @ kh[:nk].T)
         if causal:
-            S = np.where(causal_visible(sel[:, None], np.arange(nk)[None, :], Tq, Tk), S, -np.inf)
+            S = np.where(_visible(sel[:, None], np.arange(nk)[None, :], Tq, Tk, causal, window), S, -np.inf)
         lse, P = _softmax_stats(S)
         O[p0:p0 + len(sel)] = P @ vh[:nk]          # step 3: O = P V
         LSE[p0:p0 + len(sel)] = lse
     return O, LSE
 
 
-def head_backward(qh, kh, vh, doh, scale: float, causal: bool):
+def head_backward(qh, kh, vh, doh, scale: float, causal: bool, window=None):
     """One head's gradients of L = sum(dO * O) [EFF §"Real code moves even
     more", the backward products]: dV = P^T dO, dP = dO V^T,
     dS = P * (dP - D) with D_i = sum_j P_ij dP_ij, dQ = scale dS K,
-    dK = scale dS^T Q.  Returns (dQ [Tq,d], dK [Tk,d], dV [Tk,d])."""
+    dK = scale dS^T Q.  ``window`` as in head_forward.
+    Returns (dQ [Tq,d], dK [Tk,d], dV [Tk,d])."""
+    if window is not None:
+        causal = True
     Tq, Tk = qh.shape[0], kh.shape[0]
     dQ = np.zeros_like(qh)
     dK = np.zeros_like(kh)
@@ -150,7 +176,7 @@ def head_backward(qh, kh, vh, doh, scale: float, causal: bool):
         nk = _visible_keys(r1, Tq, Tk, causal)
         if nk == 0:
             continue
-        S = _masked_scores(qh[r0:r1], kh[:nk], r0, Tq, Tk, scale, causal)
+        S = _masked_scores(qh[r0:r1], kh[:nk], r0, Tq, Tk, scale, causal, window)
         _, P = _softmax_stats(S)
         dO = doh[r0:r1]
         dV[:nk] += P.T @ dO
@@ -162,9 +188,9 @@ def head_backward(qh, kh, vh, doh, scale: float, causal: bool):
     return dQ, dK, dV
 
 
-def attention_forward(q, k, v, scale: float, causal: bool):
-    """Batched, multi-head (GQA) forward over BTHD arrays.
-    Returns O [B,Tq,Hq,d] and LSE [B,Hq,Tq]."""
+def attention_forward(q, k, v, scale: float, causal: bool, window=None):
+    """Batched, multi-head (GQA) forward over BTHD arrays (``window`` as in
+    head_forward).  Returns O [B,Tq,Hq,d] and LSE [B,Hq,Tq]."""
     B, Tq, Hq, d = q.shape
     Hkv = k.shape[2]
     O = np.zeros((B, Tq, Hq, v.shape[3]))
@@ -172,11 +198,12 @@ def attention_forward(q, k, v, scale: float, causal: bool):
     for b in range(B):
         for h in range(Hq):
             g = _kv_head(h, Hq, Hkv)
-            O[b, :, h], LSE[b, h] = head_forward(q[b, :, h], k[b, :, g], v[b, :, g], scale, causal)
+            O[b, :, h], LSE[b, h] = head_forward(q[b, :, h], k[b, :, g], v[b, :, g], scale, causal,
+                                                 window=window)
     return O, LSE
 
 
-def attention_backward(q, k, v, do, scale: float, causal: bool):
+def attention_backward(q, k, v, do, scale: float, causal: bool, window=None):
     """Batched gradients; dK and dV of a KV head sum over its query heads."""
     B, Tq, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -186,16 +213,18 @@ def attention_backward(q, k, v, do, scale: float, causal: bool):
     for b in range(B):
         for h in range(Hq):
             g = _kv_head(h, Hq, Hkv)
-            a, bk, bv = head_backward(q[b, :, h], k[b, :, g], v[b, :, g], do[b, :, h], scale, causal)
+            a, bk, bv = head_backward(q[b, :, h], k[b, :, g], v[b, :, g], do[b, :, h], scale, causal, window)
             dq[b, :, h] = a
             dk[b, :, g] += bk
             dv[b, :, g] += bv
     return dq, dk, dv
 
 
-def decode_forward(q, k_cache, v_cache, seqlens, scale: float, pairs=None):
+def decode_forward(q, k_cache, v_cache, seqlens, scale: float, pairs=None, window=None):
     """One query token per sequence over the first seqlens[b] cached keys
-    [FA §"In practice", FlashDecoding]: the unmasked forward with Tq = 1.
+    [FA §"In practice", FlashDecoding]: the unmasked forward with Tq = 1 (the
+    query is the sequence's last position, so with a ``window`` it sees the
+    last ``window`` keys).
 
     q [B,Hq,d]; caches [B,Tk_max,Hkv,d].  ``pairs`` optionally restricts the
     evaluation to a list of (b, h).  Returns O [B,Hq,d], LSE [B,Hq] (entries
@@ -208,7 +237,8 @@ def decode_forward(q, k_cache, v_cache, seqlens, scale: float, pairs=None):
     for b, h in todo:
         n = int(seqlens[b])
         g = _kv_head(h, Hq, Hkv)
-        o, lse = head_forward(q[b, h][None, :], k_cache[b, :n, g], v_cache[b, :n, g], scale, False)
+        o, lse = head_forward(q[b, h][None, :], k_cache[b, :n, g], v_cache[b, :n, g], scale, False,
+                              window=window)
         O[b, h], LSE[b, h] = o[0], lse[0]
     return O, LSE
 

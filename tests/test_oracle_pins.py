@@ -350,3 +350,113 @@ def test_row_panels_do_not_change_results():
     Os, Ls = oracle.head_forward(q, k, v, 0.5, True, rows=[5, 2099, 3000 - 1000])
     np.testing.assert_array_equal(Os[1], O[2099])
     np.testing.assert_array_equal(Ls[2], LSE[2000])
+
+
+# ---------------------------------------------------------------------------
+# Sliding window (causal local window of W keys; reading of [FA "In practice"])
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("Tq,Tk,W", [(6, 6, 1), (6, 6, 3), (4, 7, 2), (5, 5, 5), (3, 8, 4)])
+def test_window_matches_brute_force(Tq, Tk, W):
+    """Each row is the softmax over exactly its W most recent visible keys,
+    computed term by term in pure Python."""
+    d = 3
+    q, k, v = _rand(1, Tq, 1, d), _rand(1, Tk, 1, d), _rand(1, Tk, 1, d)
+    s = 0.8
+    O, LSE = oracle.attention_forward(q, k, v, s, True, window=W)
+    off = Tk - Tq
+    for i in range(Tq):
+        keys = [j for j in range(Tk) if i + off - W < j <= i + off]
+        if not keys:
+            assert np.all(O[0, i, 0] == 0.0) and LSE[0, 0, i] == -np.inf
+            continue
+        scores = [s * sum(q[0, i, 0, c] * k[0, j, 0, c] for c in range(d)) for j in keys]
+        for c in range(d):
+            o, lse = oracle.brute_force_row(scores, [v[0, j, 0, c] for j in keys])
+            assert math.isclose(O[0, i, 0, c], o, rel_tol=1e-12, abs_tol=1e-13)
+        assert math.isclose(LSE[0, 0, i], lse, rel_tol=1e-13)
+
+
+def test_window_of_one_key_is_the_diagonal():
+    """W = 1: every row sees only its diagonal key, so O_i = V_{i+off},
+    LSE_i is that single score, dQ = dK = 0 and dV_j = dO of the row that sees j."""
+    Tq, Tk, d = 5, 7, 4
+    q, k, v, do = _rand(1, Tq, 2, d), _rand(1, Tk, 2, d), _rand(1, Tk, 2, d), _rand(1, Tq, 2, d)
+    s = 0.4
+    O, LSE = oracle.attention_forward(q, k, v, s, True, window=1)
+    off = Tk - Tq
+    np.testing.assert_array_equal(O[0], v[0, off:])
+    np.testing.assert_allclose(LSE[0], s * np.einsum("thd,thd->ht", q[0], k[0, off:]), rtol=1e-14)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, s, True, window=1)
+    assert np.abs(dq).max() == 0.0 and np.abs(dk).max() == 0.0
+    np.testing.assert_array_equal(dv[0, off:], do[0])
+    assert np.abs(dv[0, :off]).max() == 0.0
+
+
+def test_window_covering_all_keys_is_causal():
+    B, T, H, d = 2, 9, 2, 3
+    q, k, v, do = _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d)
+    a = oracle.attention_forward(q, k, v, 0.5, True)
+    b = oracle.attention_forward(q, k, v, 0.5, True, window=T)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+    ga = oracle.attention_backward(q, k, v, do, 0.5, True)
+    gb = oracle.attention_backward(q, k, v, do, 0.5, True, window=T + 3)
+    for x, y in zip(ga, gb):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_window_row_equals_unmasked_attention_over_its_slice():
+    """A windowed row is plain (unmasked) attention over the key slice
+    [i + off - W + 1, i + off]."""
+    Tq, Tk, d, W = 40, 50, 3, 7
+    q, k, v = _rand(Tq, d), _rand(Tk, d), _rand(Tk, d)
+    O, LSE = oracle.head_forward(q, k, v, 0.3, True, window=W)
+    off = Tk - Tq
+    for i in (0, 1, 13, 39):
+        lo, hi = max(0, i + off - W + 1), i + off + 1
+        Oi, Li = oracle.head_forward(q[i:i + 1], k[lo:hi], v[lo:hi], 0.3, False)
+        np.testing.assert_allclose(O[i], Oi[0], rtol=1e-13, atol=1e-15)
+        assert math.isclose(LSE[i], Li[0], rel_tol=1e-14)
+
+
+def test_window_backward_finite_differences():
+    B, T, H, d, W = 1, 7, 1, 3, 3
+    q, k, v, do = _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d), _rand(B, T, H, d)
+    s = 0.6
+
+    def loss(q_, k_, v_):
+        return float((oracle.attention_forward(q_, k_, v_, s, True, window=W)[0] * do).sum())
+
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, s, True, window=W)
+    eps = 1e-5
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            args_p = {"q_": q, "k_": k, "v_": v}
+            args_m = dict(args_p)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p[name + "_"], args_m[name + "_"] = xp, xm
+            num[idx] = (loss(**args_p) - loss(**args_m)) / (2 * eps)
+        rel = np.linalg.norm(num - g) / np.linalg.norm(g)
+        assert rel <= 1e-6, (name, rel)
+
+
+def test_window_decode_is_last_prefill_row():
+    """Decode with a window sees the last W keys of the sequence, i.e. the
+    last row of a windowed prefill over the prefix."""
+    B, Hq, Hkv, d, Tmax, W = 3, 4, 2, 3, 30, 5
+    q = _rand(B, Hq, d)
+    kc, vc = _rand(B, Tmax, Hkv, d), _rand(B, Tmax, Hkv, d)
+    seqlens = [2, 11, 30]
+    O, LSE = oracle.decode_forward(q, kc, vc, seqlens, 0.3, window=W)
+    for b in range(B):
+        n = seqlens[b]
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            lo = max(0, n - W)
+            Ob, Lb = oracle.head_forward(q[b, h][None, :], kc[b, lo:n, g], vc[b, lo:n, g], 0.3, False)
+            np.testing.assert_allclose(O[b, h], Ob[0], rtol=1e-13, atol=1e-15)
+            assert math.isclose(LSE[b, h], Lb[0], rel_tol=1e-14)

@@ -50,13 +50,24 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--window", type=int, default=None,
+                    help="sliding window of that many keys on a prefill workload (implies causal)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (smaller cases for profiler captures only)")
     return ap.parse_args()
 
 
-def pairs_count(Tq, Tk, causal):
-    """(query, key) pairs entering the softmax; bottom-right causal rule."""
+def pairs_count(Tq, Tk, causal, window=0):
+    """(query, key) pairs entering the softmax; bottom-right causal rule, and
+    with a sliding window the `window` most recent keys of each query."""
+    if window:
+        off = Tk - Tq
+        tot = 0
+        for i in range(Tq):
+            hi = min(Tk - 1, i + off)
+            lo = max(0, i + off - window + 1)
+            tot += max(0, hi - lo + 1)
+        return tot
     if not causal:
         return Tq * Tk
     off = Tk - Tq
@@ -70,7 +81,7 @@ def pairs_count(Tq, Tk, causal):
 
 
 def flops(w):
-    P = pairs_count(w.T, w.T, w.causal)
+    P = pairs_count(w.T, w.T, w.causal, w.window)
     f = 4 * w.B * w.Hq * w.d * P
     b = 10 * w.B * w.Hq * w.d * P
     return f, b
@@ -194,8 +205,9 @@ def oracle_heads(w, inp_cpu, heads, budget_s):
         kh = to_f64(inp_cpu["k"][bi, :, g])
         vh = to_f64(inp_cpu["v"][bi, :, g])
         dh = to_f64(inp_cpu["do"][bi, :, h])
-        oracle.head_forward(qh, kh, vh, w.scale, w.causal)
-        oracle.head_backward(qh, kh, vh, dh, w.scale, w.causal)
+        win = w.window or None
+        oracle.head_forward(qh, kh, vh, w.scale, w.causal, window=win)
+        oracle.head_backward(qh, kh, vh, dh, w.scale, w.causal, window=win)
         done += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -237,7 +249,8 @@ def run_reference(args, w, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d,
-                   "causal": w.causal, "step": "one head of the workload, forward + backward"},
+                   "causal": w.causal, "window": w.window or None,
+                   "step": "one head of the workload, forward + backward"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": f"one (batch, head) of {w.name} per step, float64 numpy"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -294,6 +307,11 @@ def run_fa(args, w, rank, world, dist):
     stream = torch.cuda.current_stream(dev)
     sp = P(stream.cuda_stream)
     scale, causal = w.scale, int(w.causal)
+    # with a sliding window the windowed entry points take the window in
+    # place of the causal flag
+    fwd_fn, dkdv_fn, mask_arg = lib.fa_forward, lib.fa_backward_dkdv, causal
+    if w.window:
+        fwd_fn, dkdv_fn, mask_arg = lib.fa_forward_window, lib.fa_backward_dkdv_window, w.window
 
     def check(st, name):
         if st != 0:
@@ -301,12 +319,12 @@ def run_fa(args, w, rank, world, dist):
 
     def step(evs=None):
         if evs: evs[0].record(stream)
-        check(lib.fa_forward(pq, pk, pv, po, plse, B, Hq, Hkv, T, T, d, scale, causal, sp), "fa_forward")
+        check(fwd_fn(pq, pk, pv, po, plse, B, Hq, Hkv, T, T, d, scale, mask_arg, sp), "fa_forward")
         if evs: evs[1].record(stream)
         check(lib.fa_backward_preprocess(po, plse, pdo, pws, ws_bytes, B, Hq, Hkv, T, T, d, sp), "preprocess")
         if evs: evs[2].record(stream)
-        check(lib.fa_backward_dkdv(pq, pk, pv, pdo, pdk, pdv, pws, ws_bytes, B, Hq, Hkv, T, T, d, scale, causal,
-                                   sp), "dkdv")
+        check(dkdv_fn(pq, pk, pv, pdo, pdk, pdv, pws, ws_bytes, B, Hq, Hkv, T, T, d, scale, mask_arg, sp),
+              "dkdv")
         if evs: evs[3].record(stream)
         check(lib.fa_backward_dq_finalize(pdq, pws, ws_bytes, B, Hq, Hkv, T, T, d, sp), "dq_finalize")
         if evs: evs[4].record(stream)
@@ -390,8 +408,10 @@ def run_fa(args, w, rank, world, dist):
         def e2e_step():
             q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True); do.copy_(hdo, non_blocking=True)
-            fa.forward(q, k, v, scale=scale, causal=w.causal, out=o, lse=lse)
-            fa.backward(q, k, v, o, lse, do, scale=scale, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+            win = w.window or None
+            fa.forward(q, k, v, scale=scale, causal=w.causal, out=o, lse=lse, window=win)
+            fa.backward(q, k, v, o, lse, do, scale=scale, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv,
+                        window=win)
             ho.copy_(o, non_blocking=True); hlse.copy_(lse, non_blocking=True)
             hdq.copy_(dq, non_blocking=True); hdk.copy_(dk, non_blocking=True); hdv.copy_(dv, non_blocking=True)
 
@@ -421,6 +441,7 @@ def run_fa(args, w, rank, world, dist):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
+                       "window": w.window or None,
                        "step": "fa_forward + fa_backward (preprocess, dkdv, dq_finalize)",
                        "l2": "inputs larger than L2 (q, k, v, dO: 4 x %d MiB per step)" % (q.numel() * 2 >> 20),
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -521,6 +542,11 @@ def main():
     w = WORKLOADS[args.workload]
     if args.batch is not None:
         w = w.with_(B=args.batch)
+    if args.window is not None:
+        if w.decode or args.window < 1:
+            print("--window applies to the prefill workloads and must be >= 1", file=sys.stderr)
+            return 2
+        w = w.with_(window=args.window, causal=True)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     dist = None

@@ -85,6 +85,20 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
                void* stream);
 
 /*
+ * fa_forward_window -- fa_forward with a sliding-window mask: query i sees
+ * key j iff i + (Tk - Tq) - window < j <= i + (Tk - Tq), i.e. its own
+ * (bottom-right aligned) diagonal key and the window - 1 keys before it.
+ * ("FlashAttention", "In practice", names sliding windows next to GQA and
+ * causal masks without defining them; this causal local window is the
+ * reading used here.)  window >= Tk gives the causal result; window < 1 or
+ * above 2^30 is FA_ERR_INVALID_ARG.  Other arguments as fa_forward.  Key
+ * tiles wholly outside every window of a query tile are not read.
+ */
+int fa_forward_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int window,
+                      void* stream);
+
+/*
  * Bytes of device workspace fa_backward needs: an fp32 dQ accumulator
  * [B,Tq,Hq,d], the fp32 row terms D_i = sum_c dO_ic O_ic and the LSE in log2
  * units, each [B,Hq,Tq_pad] with Tq_pad = Tq rounded up to 128; every piece
@@ -111,6 +125,17 @@ int fa_backward(const void* q, const void* k, const void* v, const void* o,
                 void* stream);
 
 /*
+ * fa_backward_window -- gradients of fa_forward_window (same window rule;
+ * o and lse must come from fa_forward_window with the same window).  Other
+ * arguments, the workspace and the errors as fa_backward.
+ */
+int fa_backward_window(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                       void* ws, size_t ws_bytes,
+                       int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int window,
+                       void* stream);
+
+/*
  * The three steps fa_backward runs, in this order on one stream, exposed so
  * that a caller can schedule or time them separately.  They share the
  * workspace of fa_backward_workspace_bytes() and its layout; arguments mean
@@ -128,6 +153,12 @@ int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void
 int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
                      void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d,
                      float scale, int causal, void* stream);
+
+/* fa_backward_dkdv with the sliding window of fa_forward_window (window >= 1). */
+int fa_backward_dkdv_window(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                            void* dv, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq,
+                            int Tk, int d, float scale, int window, void* stream);
+
 int fa_backward_dq_finalize(void* dq, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk,
                             int d, void* stream);
 

@@ -32,10 +32,13 @@ SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_version": (_c_int, []),
     "fa_forward": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_forward_window": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_workspace_bytes": (_c_size, [_c_int] * 6),
     "fa_backward": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_backward_window": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_preprocess": (_c_int, [_vp] * 4 + [_c_size] + [_c_int] * 6 + [_vp]),
     "fa_backward_dkdv": (_c_int, [_vp] * 7 + [_c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_backward_dkdv_window": (_c_int, [_vp] * 7 + [_c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_dq_finalize": (_c_int, [_vp] * 2 + [_c_size] + [_c_int] * 6 + [_vp]),
     "fa_decode_workspace_bytes": (_c_size, [_c_int] * 5),
     "fa_decode_splitkv": (_c_int, [_vp] * 6 + [_vp, _c_size] + [_c_int] * 5 + [_c_float, _c_int, _vp]),
@@ -98,8 +101,10 @@ def _raise(fn, st):
         raise FAError(fn, st)
 
 
-def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
-    """O, LSE = attention(q, k, v).  q [B,Tq,Hq,d], k/v [B,Tk,Hkv,d] bf16 (CUDA)."""
+def forward(q, k, v, scale=None, causal=False, out=None, lse=None, window=None):
+    """O, LSE = attention(q, k, v).  q [B,Tq,Hq,d], k/v [B,Tk,Hkv,d] bf16 (CUDA).
+    ``window`` (int >= 1) selects the sliding-window mask of fa_forward_window
+    (which includes the causal one)."""
     lib = load_library()
     B, Tq, Hq, d = q.shape
     Tk, Hkv = k.shape[1], k.shape[2]
@@ -114,9 +119,14 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
         lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=dev)
     _check_dev("out", out, torch.bfloat16, dev)
     _check_dev("lse", lse, torch.float32, dev)
-    st = lib.fa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tk, d,
-                        float(scale), int(bool(causal)), _stream_ptr(dev))
-    _raise("fa_forward", st)
+    if window is None:
+        st = lib.fa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tk, d,
+                            float(scale), int(bool(causal)), _stream_ptr(dev))
+        _raise("fa_forward", st)
+    else:
+        st = lib.fa_forward_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tk, d,
+                                   float(scale), int(window), _stream_ptr(dev))
+        _raise("fa_forward_window", st)
     return out, lse
 
 
@@ -124,9 +134,10 @@ def backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d) -> int:
     return int(load_library().fa_backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d))
 
 
-def backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None, dq=None, dk=None, dv=None):
+def backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None, dq=None, dk=None, dv=None,
+             window=None):
     """dQ, dK, dV for L = sum(dO * O).  `workspace` (uint8 CUDA tensor) is
-    allocated here when not given."""
+    allocated here when not given; ``window`` as in forward()."""
     lib = load_library()
     B, Tq, Hq, d = q.shape
     Tk, Hkv = k.shape[1], k.shape[2]
@@ -142,10 +153,14 @@ def backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None, dq=N
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    st = lib.fa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
-                         _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tq, Tk, d,
-                         float(scale), int(bool(causal)), _stream_ptr(dev))
-    _raise("fa_backward", st)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+            _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tq, Tk, d, float(scale))
+    if window is None:
+        st = lib.fa_backward(*args, int(bool(causal)), _stream_ptr(dev))
+        _raise("fa_backward", st)
+    else:
+        st = lib.fa_backward_window(*args, int(window), _stream_ptr(dev))
+        _raise("fa_backward_window", st)
     return dq, dk, dv
 
 

@@ -198,10 +198,14 @@ const char* fa_status_string(int s) {
 
 int fa_version(void) { return 100; }
 
-int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-               int Hkv, int Tq, int Tk, int d, float scale, int causal, void* stream) {
+}  // extern "C"
+
+// window > 0: sliding window of that many keys (the caller passes causal = 1).
+static int forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                        int Hkv, int Tq, int Tk, int d, float scale, int causal, int window, void* stream) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
+  if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
   if (B == 0 || Tq == 0) return FA_OK;
   if (!q || !o || !lse || (Tk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || (Tk > 0 && (!aligned16(k) || !aligned16(v))))
@@ -218,6 +222,7 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
   p.lse = lse;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tq = Tq; p.Tk = Tk;
   p.causal = causal;
+  p.window = window;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_mblocks = (Tq + 255) / 256;
   p.n_items = B * Hq * p.n_mblocks;
@@ -234,6 +239,19 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
   else
     fa_fwd_kernel<128><<<grid, FwdCfg<128>::THREADS, FwdCfg<128>::SMEM_BYTES, s>>>(p);
   return launch_status();
+}
+
+extern "C" {
+
+int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Tq, int Tk, int d, float scale, int causal, void* stream) {
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0, stream);
+}
+
+int fa_forward_window(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                      int Hkv, int Tq, int Tk, int d, float scale, int window, void* stream) {
+  if (window < 1) return FA_ERR_INVALID_ARG;
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, d, scale, 1, window, stream);
 }
 
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -296,11 +314,14 @@ int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void
   return launch_status();
 }
 
-int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
-                     void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d,
-                     float scale, int causal, void* stream) {
+}  // extern "C"
+
+static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* ws,
+                     size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal,
+                     int window, void* stream) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
+  if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
   if (B == 0 || Tk == 0) return FA_OK;
   if ((st = check_ptrs({k, v, dk, dv}))) return st;
   if (Tq > 0 && (st = check_ptrs({q, dO}))) return st;
@@ -323,6 +344,7 @@ int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO
   p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
   p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tq = Tq; p.Tk = Tk; p.causal = causal;
+  p.window = window;
   p.Tq_pad = tq_pad(Tq);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -346,6 +368,21 @@ int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO
   return launch_status();
 }
 
+extern "C" {
+
+int fa_backward_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                     void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+                     float scale, int causal, void* stream) {
+  return dkdv_impl(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0, stream);
+}
+
+int fa_backward_dkdv_window(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                            void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+                            float scale, int window, void* stream) {
+  if (window < 1) return FA_ERR_INVALID_ARG;
+  return dkdv_impl(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, 1, window, stream);
+}
+
 int fa_backward_dq_finalize(void* dq, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk,
                             int d, void* stream) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, 1.f, 0);
@@ -361,19 +398,39 @@ int fa_backward_dq_finalize(void* dq, void* ws, size_t ws_bytes, int B, int Hq, 
   return launch_status();
 }
 
-int fa_backward(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B,
-                int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal, void* stream) {
+}  // extern "C"
+
+static int backward_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B, int Hq,
+                         int Hkv, int Tq, int Tk, int d, float scale, int causal, int window, void* stream) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
+  if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
   if (B == 0 || (Tq == 0 && Tk == 0)) return FA_OK;
   if (Tq > 0 && (st = check_ptrs({q, o, lse, dO, dq}))) return st;
   if (Tk > 0 && (st = check_ptrs({k, v, dk, dv}))) return st;
   if ((st = check_ws(ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d))) return st;
   if ((st = fa_backward_preprocess(o, lse, dO, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream))) return st;
-  if ((st = fa_backward_dkdv(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, stream)))
+  if ((st = dkdv_impl(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, window, stream)))
     return st;
   return fa_backward_dq_finalize(dq, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream);
+}
+
+extern "C" {
+
+int fa_backward(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B,
+                int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal, void* stream) {
+  return backward_impl(q, k, v, o, lse, dO, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0,
+                       stream);
+}
+
+int fa_backward_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B,
+                       int Hq, int Hkv, int Tq, int Tk, int d, float scale, int window, void* stream) {
+  if (window < 1) return FA_ERR_INVALID_ARG;
+  return backward_impl(q, k, v, o, lse, dO, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, 1, window,
+                       stream);
 }
 
 static size_t decode_nchunk(int Tk_max, int chunk) { return ((size_t)Tk_max + chunk - 1) / chunk; }

@@ -130,6 +130,7 @@ struct BwdParams {
   __nv_bfloat16* dk;   // [B][Tk][Hkv][d]
   __nv_bfloat16* dv;
   int B, Hq, Hkv, Tq, Tk, causal;
+  int window;          // > 0: sliding window of that many keys (implies causal)
   int Tq_pad;          // row pitch of lse2 / Dv
   float scale, scale_log2;
   int n_kv_tiles;
@@ -225,11 +226,17 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   it.j0 = kt * 128;
   const int n_qt = (p.Tq + 127) / 128;
   it.qt_begin = 0;
+  int qt_end = n_qt;
   if (p.causal) {
     const int qmin = it.j0 - (p.Tk - p.Tq);   // first query that sees key j0
     it.qt_begin = qmin <= 0 ? 0 : min(n_qt, qmin / 128);
+    if (p.window > 0) {
+      // last query whose window still holds the tile's last key
+      const long long qmax = (long long)it.j0 + 127 - (p.Tk - p.Tq) + p.window - 1;
+      qt_end = qmax < 0 ? 0 : (int)min((long long)n_qt, qmax / 128 + 1);
+    }
   }
-  it.nq = n_qt - it.qt_begin;
+  it.nq = max(0, qt_end - it.qt_begin);
   it.n_it = (p.Hq / p.Hkv) * it.nq;
   return it;
 }
@@ -518,7 +525,9 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         tc_fence_after();
         const float* lrow = lse_s + s * 128 + 64 * half;
         const int cmin = p.causal ? qmin - q0 - 64 * half : 0;  // columns < cmin are masked
-        const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > 0);
+        // and, with a window, columns >= cmax (queries past this key's window)
+        const int cmax = p.window > 0 ? qmin + p.window - q0 - 64 * half : (1 << 30);
+        const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > 0 || cmax < 64);
         // 64 query columns in four 16-column chunks; the load of chunk c+1
         // overlaps the exponentials of chunk c.  P^T (bf16 pairs) goes to
         // the first 32 columns of this warp's 64, never ahead of its loads.
@@ -539,8 +548,8 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             float p0 = ex2_approx(x.x);
             float p1 = ex2_approx(x.y);
             if (masked) {
-              if (!key_ok || col < cmin) p0 = 0.f;
-              if (!key_ok || col + 1 < cmin) p1 = 0.f;
+              if (!key_ok || col < cmin || col >= cmax) p0 = 0.f;
+              if (!key_ok || col + 1 < cmin || col + 1 >= cmax) p1 = 0.f;
             }
             pk[e] = pack_bf16x2(p0, p1);
           }
@@ -641,23 +650,21 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             const float2 r = __fmul2_rn(pf, t);
             pp[8 * c + e] = pack_bf16x2(r.x, r.y);
           }
-          if (c == 0 && gi > 0) {
-            // The shared dS tile is still an operand of the previous tile's
-            // dK and dQ MMAs until they complete (this tile's dP^T can
-            // complete before them).
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
-            if (!ok) break;
-          }
-          // dS into shared memory: row j of box `half`, 16-byte chunks 2c and
-          // 2c+1, 128-byte swizzle (chunk ^ (row % 8)).
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int chunk = 2 * c + q;
-            *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (j & 7)) << 4)) =
-                make_uint4(pp[8 * c + 4 * q], pp[8 * c + 4 * q + 1], pp[8 * c + 4 * q + 2], pp[8 * c + 4 * q + 3]);
-          }
         }
+        if (gi > 0) {
+          // The shared dS tile is still an operand of the previous tile's
+          // dK and dQ MMAs until they complete (this tile's dP^T can
+          // complete before them); the arithmetic above overlaps that wait.
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
+          if (!ok) break;
+        }
+        // dS into shared memory: row j of box `half`, eight 16-byte chunks,
+        // 128-byte swizzle (chunk ^ (row % 8)).
+#pragma unroll
+        for (int chunk = 0; chunk < 8; ++chunk)
+          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (j & 7)) << 4)) =
+              make_uint4(pp[4 * chunk], pp[4 * chunk + 1], pp[4 * chunk + 2], pp[4 * chunk + 3]);
         if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_before();

@@ -1,5 +1,9 @@
-// fa_fwd.cuh -- forward kernel: O = softmax(scale QK^T [+ causal mask]) V and
-// one fp32 log-sum-exp per row, tile by tile with the online softmax.
+// fa_fwd.cuh -- forward kernel: O = softmax(scale QK^T [+ causal or
+// sliding-window mask]) V and one fp32 log-sum-exp per row, tile by tile with
+// the online softmax.  (The sliding window, named next to GQA in the
+// "FlashAttention" interview track's "In practice" section, is read as a
+// causal window of the W most recent keys; tiles wholly outside it are not
+// loaded.)
 //
 // Method: "Flash Attention: Why Memory Traffic, Not Compute, Is the
 // Bottleneck", sections "Flash Attention Uses Tiles" (Q/K/V tiles in on-chip
@@ -45,6 +49,7 @@ struct FwdParams {
   float* lse;         // [B][Hq][Tq]
   int B, Hq, Hkv, Tq, Tk;
   int causal;
+  int window;         // > 0: sliding window of that many keys (implies causal)
   float scale_log2;   // scale * log2(e)
   int n_mblocks;      // ceil(Tq / 256): work items per (batch, head)
   int n_items;        // B * Hq * n_mblocks
@@ -79,9 +84,10 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
 };
 
-// One work item: two query tiles [m0, m0 + 256) of head h of batch b.
+// One work item: two query tiles [m0, m0 + 256) of head h of batch b,
+// against KV tiles kv0 .. kv0 + n_kv - 1.
 struct FwdItem {
-  int b, h, hkv, m0, n_kv;
+  int b, h, hkv, m0, kv0, n_kv;
 };
 
 template <int D>
@@ -97,11 +103,19 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   it.hkv = it.h / (p.Hq / p.Hkv);
   it.m0 = (p.n_mblocks - 1 - item % p.n_mblocks) * 2 * C::BM;
   const int n_kv_all = (p.Tk + C::BN - 1) / C::BN;
+  it.kv0 = 0;
   it.n_kv = n_kv_all;
   if (p.causal) {
     const int last_row = min(it.m0 + 2 * C::BM, p.Tq) - 1;
     const int kmax = last_row + (p.Tk - p.Tq);  // last visible key (inclusive)
     it.n_kv = kmax < 0 ? 0 : min(n_kv_all, kmax / C::BN + 1);
+    if (p.window > 0) {
+      // the first row's window starts at its first visible key; tiles
+      // before it are skipped
+      const int kmin = it.m0 + (p.Tk - p.Tq) - p.window + 1;
+      it.kv0 = kmin <= 0 ? 0 : min(it.n_kv, kmin / C::BN);
+      it.n_kv -= it.kv0;
+    }
   }
   return it;
 }
@@ -186,7 +200,8 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
             mbar_arrive_expect_tx(bar_kv_full(s), C::TILE_BYTES);
             const CUtensorMap* tm = which ? &p.tm_v : &p.tm_k;
             for (int kb = 0; kb < C::NBOX; ++kb)
-              tma_load_4d(stage_addr(s) + kb * C::BOX_BYTES, tm, bar_kv_full(s), kb * 64, it.hkv, j * C::BN, it.b);
+              tma_load_4d(stage_addr(s) + kb * C::BOX_BYTES, tm, bar_kv_full(s), kb * 64, it.hkv,
+                          (it.kv0 + j) * C::BN, it.b);
           }
         }
         ++qi;
@@ -284,6 +299,7 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
       const FwdItem it = fwd_item<D>(p, item);
       const int row = it.m0 + w * C::BM + r;
       const int key_limit = p.causal ? min(p.Tk, row + (p.Tk - p.Tq) + 1) : p.Tk;  // keys < limit visible
+      const int key_lo = p.window > 0 ? row + (p.Tk - p.Tq) - p.window + 1 : 0;     // and keys >= key_lo
       float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
       float l = 0.f;
       for (int j = 0; j < it.n_kv; ++j) {
@@ -294,11 +310,13 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, su + c * 32);
         tmem_wait_ld();
-        const int nvalid = key_limit - j * C::BN;
-        if (__any_sync(0xffffffffu, nvalid < C::BN)) {
+        const int nvalid = key_limit - (it.kv0 + j) * C::BN;  // columns >= nvalid are masked
+        const int nlo = key_lo - (it.kv0 + j) * C::BN;         // and columns < nlo
+        const bool masked = __any_sync(0xffffffffu, nvalid < C::BN || nlo > 0);
+        if (masked) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (c >= nvalid) su[c] = __float_as_uint(-INFINITY);
+            if (c >= nvalid || c < nlo) su[c] = __float_as_uint(-INFINITY);
         }
         // Row maximum: eight independent chains, then a short tree.
         float mx8[8];
@@ -324,7 +342,6 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
         const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nref = make_float2(-ref, -ref);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        const bool masked = __any_sync(0xffffffffu, nvalid < C::BN);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(su[2 * c]), __uint_as_float(su[2 * c + 1])), sl2, nref);
@@ -332,8 +349,8 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
           // unit, shared by both softmax warpgroups, is not the bottleneck.
           float2 pr = C::poly_pair(c) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
           if (C::poly_pair(c) && masked) {
-            if (2 * c >= nvalid) pr.x = 0.f;
-            if (2 * c + 1 >= nvalid) pr.y = 0.f;
+            if (2 * c >= nvalid || 2 * c < nlo) pr.x = 0.f;
+            if (2 * c + 1 >= nvalid || 2 * c + 1 < nlo) pr.y = 0.f;
           }
           acc[c & 3] = __fadd2_rn(acc[c & 3], pr);
           su[c] = pack_bf16x2(pr.x, pr.y);

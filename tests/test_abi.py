@@ -99,3 +99,15 @@ def test_product_path_has_no_oracle_dependency():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower() or f.endswith((".cu", ".cuh", ".h")) and "oracle" not in text, f
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_window_entry_points_reject_bad_window_on_host():
+    lib = fa.load_library()
+    # window must be >= 1 (and at most 2^30); checked before any pointer
+    for w in (0, -3, (1 << 30) + 1):
+        assert lib.fa_forward_window(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 16, 16, 64, 1.0, w, NULL) == 1
+        assert lib.fa_backward_window(*([NULL] * 9), NULL, 0, 1, 1, 1, 16, 16, 64, 1.0, w, NULL) == 1
+    # a valid window with null pointers is still rejected; empty query is a no-op
+    assert lib.fa_forward_window(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 16, 16, 64, 1.0, 4, NULL) == 1
+    assert lib.fa_forward_window(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 0, 16, 64, 1.0, 4, NULL) == 0
+    assert lib.fa_forward_window(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 16, 16, 96, 1.0, 4, NULL) == 2

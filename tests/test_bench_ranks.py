@@ -54,3 +54,6 @@ def test_pair_count_matches_brute_force():
         for causal in (False, True):
             brute = sum(1 for i in range(Tq) for j in range(Tk) if (not causal) or j <= i + Tk - Tq)
             assert bench.pairs_count(Tq, Tk, causal) == brute
+        for W in (1, 2, 7, 128, 1000):
+            brute = sum(1 for i in range(Tq) for j in range(Tk) if i + Tk - Tq - W < j <= i + Tk - Tq)
+            assert bench.pairs_count(Tq, Tk, True, W) == brute

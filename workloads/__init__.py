@@ -52,6 +52,7 @@ class Workload:
     tk_lo: int = 0
     tk_hi: int = 0
     chunk: int = 256
+    window: int = 0   # > 0: sliding window of that many keys (implies causal)
 
     @property
     def scale(self) -> float:

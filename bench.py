@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--window", type=int, default=None,
-                    help="sliding window of that many keys on a prefill workload (implies causal)")
+                    help="sliding window of that many keys (prefill: implies causal; decode: last keys)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (smaller cases for profiler captures only)")
     return ap.parse_args()
@@ -215,6 +215,28 @@ def oracle_heads(w, inp_cpu, heads, budget_s):
     return done, dt, done * per_head
 
 
+def oracle_decode(w, q, kc, vc, seqlens, budget_s):
+    """Run the oracle's decode (G query heads of one KV head at a time) over
+    the given sequences; stop at the budget.  Returns (groups done, seconds,
+    algorithmic bytes done: the K and V rows the query sees, q, o, lse)."""
+    import oracle
+    from workloads import to_f64
+    G = w.Hq // w.Hkv
+    done, nbytes, t0 = 0, 0, time.perf_counter()
+    while True:   # passes over the given sequences until the budget is spent
+        for b in range(q.shape[0]):
+            L = int(seqlens[b])
+            seen = min(L, w.window) if w.window else L
+            qb, kb, vb = to_f64(q[b:b + 1]), to_f64(kc[b:b + 1, :L]), to_f64(vc[b:b + 1, :L])
+            for hkv in range(w.Hkv):
+                oracle.decode_forward(qb, kb, vb, [L], w.scale, pairs=[(0, hkv * G + i) for i in range(G)],
+                                      window=w.window or None)
+                done += 1
+                nbytes += seen * w.d * 2 * 2 + G * (w.d * 2 * 2 + 4)
+                if time.perf_counter() - t0 >= budget_s:
+                    return done, time.perf_counter() - t0, nbytes
+
+
 def cpu_baseline(w, inp_cpu, budget_s):
     heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
     done, dt, fl = oracle_heads(w, inp_cpu, heads, budget_s)
@@ -227,12 +249,50 @@ def cpu_baseline(w, inp_cpu, budget_s):
 # reference arm
 # ---------------------------------------------------------------------------
 
+def run_reference_decode(args, w):
+    """The oracle's decode on the host cores: each step one (sequence, KV
+    head) group of two sequences drawn like the workload's."""
+    from workloads import decode_inputs
+    inp = decode_inputs(w.with_(B=2), device="cpu")
+    q, kc, vc, sl = inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"]
+    G = w.Hq // w.Hkv
+    groups = [(b, hkv) for b in range(2) for hkv in range(w.Hkv)]
+
+    def one(s):
+        b, hkv = groups[s % len(groups)]
+        sub = w.with_(Hq=G, Hkv=1)
+        return oracle_decode(sub, q[b:b + 1, hkv * G:(hkv + 1) * G], kc[b:b + 1, :, hkv:hkv + 1],
+                             vc[b:b + 1, :, hkv:hkv + 1], sl[b:b + 1], 1e9)
+
+    for s in range(args.warmup):
+        one(s)
+    tot_b, tot_t = 0, 0.0
+    for s in range(args.steps):
+        _, dt, nb = one(s)
+        tot_b += nb
+        tot_t += dt
+    value = tot_b / tot_t / 1e9
+    line = {
+        "impl": "reference", "metric": "split-KV decode HBM GB/s (bf16 KV cache, 1xB200) and % of HBM peak",
+        "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Tk_max": w.T, "d": w.d,
+                   "chunk": w.chunk, "window": w.window or None,
+                   "step": "one (sequence, KV head) group of the workload"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one (sequence, KV head) group of {w.name} per step, float64 numpy"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return 0
     if w.decode:
-        print(json.dumps({"impl": "reference", "unavailable": "reference arm covers the prefill workloads"}))
-        return 0
+        return run_reference_decode(args, w)
     from workloads import prefill_inputs
     inp = prefill_inputs(w.with_(B=1), device="cpu")
     heads = [(0, h) for h in range(w.Hq)]
@@ -482,14 +542,20 @@ def run_decode(args, w, rank, world, dist):
     stream = torch.cuda.current_stream(dev)
     sp = P(stream.cuda_stream)
     args_c = (P(q.data_ptr()), P(kc.data_ptr()), P(vc.data_ptr()), P(sl.data_ptr()), P(o.data_ptr()),
-              P(lse.data_ptr()), P(ws.data_ptr()), wsb, B, Hq, Hkv, Tk_max, d, w.scale, chunk, sp)
+              P(lse.data_ptr()), P(ws.data_ptr()), wsb, B, Hq, Hkv, Tk_max, d, w.scale, chunk)
+    dec_fn = lib.fa_decode_splitkv
+    if w.window:
+        dec_fn = lib.fa_decode_splitkv_window
+        args_c = args_c + (w.window,)
+    args_c = args_c + (sp,)
 
     def step():
-        st = lib.fa_decode_splitkv(*args_c)
+        st = dec_fn(*args_c)
         if st != 0:
             raise RuntimeError(f"fa_decode_splitkv: {fa.STATUS.get(st, st)}")
 
-    total_keys = int(sl.sum().item())
+    # keys the query sees: the whole prefix, or its last `window` keys
+    total_keys = int(sl.clamp(max=w.window).sum().item()) if w.window else int(sl.sum().item())
     alg_bytes = total_keys * Hkv * d * 2 * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
 
     def barrier():
@@ -516,6 +582,14 @@ def run_decode(args, w, rank, world, dist):
     value = job_rate(alg_bytes, world, args.steps, ms) / 1e9
     peaks = load_peaks()
     # dominant kernel time: split kernel alone, timed separately on the same stream
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle over the first two sequences' caches, copied to the host
+        nb, dt, nbytes = oracle_decode(w, q[:2].cpu(), kc[:2].cpu(), vc[:2].cpu(), sl[:2].cpu(), args.cpu_seconds)
+        cpu = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"float64 oracle decode of {nb} (sequence, KV head) groups, cycling over the first two "
+                         f"sequences of {w.name} ({dt:.1f} s; same algorithmic bytes as the GPU metric)"}
+
     if rank == 0:
         line = {
             "metric": "split-KV decode HBM GB/s (bf16 KV cache, 1xB200) and % of HBM peak",
@@ -523,14 +597,16 @@ def run_decode(args, w, rank, world, dist):
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "Tk_max": Tk_max, "d": d, "chunk": chunk,
-                       "total_cached_tokens": total_keys, "l2": "KV cache larger than L2", "seed": w.seed},
+                       "total_cached_tokens": total_keys, "window": w.window or None,
+                       "l2": "KV cache larger than L2", "seed": w.seed},
             "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_combine_kernel", "bound": "hbm",
                          "achieved": value / world, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": value / world / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy",
                          "traffic": traffic_from_profile("fa_decode_split_kernel", w.name),
                          "algorithmic_per_launch": alg_bytes},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": 3 * args.steps,   # split, combine, empty-sequence kernels
             "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -543,10 +619,10 @@ def main():
     if args.batch is not None:
         w = w.with_(B=args.batch)
     if args.window is not None:
-        if w.decode or args.window < 1:
-            print("--window applies to the prefill workloads and must be >= 1", file=sys.stderr)
+        if args.window < 1:
+            print("--window must be >= 1", file=sys.stderr)
             return 2
-        w = w.with_(window=args.window, causal=True)
+        w = w.with_(window=args.window, causal=not w.decode)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     dist = None

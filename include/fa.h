@@ -187,6 +187,18 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
                       void* stream);
 
 /*
+ * fa_decode_splitkv_window -- fa_decode_splitkv with the sliding window of
+ * fa_forward_window: the query (the sequence's last position) sees only the
+ * last `window` cached keys, min(window, seqlens_k[b]) of them.  Chunks that
+ * hold none of them are skipped.  window >= 1; other arguments, workspace
+ * and errors as fa_decode_splitkv.
+ */
+int fa_decode_splitkv_window(const void* q, const void* k_cache, const void* v_cache,
+                             const int* seqlens_k, void* o, float* lse, void* ws, size_t ws_bytes,
+                             int B, int Hq, int Hkv, int Tk_max, int d, float scale, int chunk,
+                             int window, void* stream);
+
+/*
  * fa_decode_splitkv_noalloc -- fa_decode_splitkv for callers that cannot
  * allocate device memory where they call it: code running inside a CUDA
  * graph capture or a plug-in interface that only hands over inputs and

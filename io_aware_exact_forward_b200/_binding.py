@@ -42,6 +42,8 @@ SIGNATURES = {
     "fa_backward_dq_finalize": (_c_int, [_vp] * 2 + [_c_size] + [_c_int] * 6 + [_vp]),
     "fa_decode_workspace_bytes": (_c_size, [_c_int] * 5),
     "fa_decode_splitkv": (_c_int, [_vp] * 6 + [_vp, _c_size] + [_c_int] * 5 + [_c_float, _c_int, _vp]),
+    "fa_decode_splitkv_window": (_c_int, [_vp] * 6 + [_vp, _c_size] + [_c_int] * 5 + [_c_float, _c_int, _c_int,
+                                                                                    _vp]),
     "fa_decode_splitkv_noalloc": (_c_int, [_vp] * 6 + [_c_int] * 5 + [_c_float, _c_int, _vp]),
     "fa_check": (_c_int, [_vp]),
     "fa_selftest_bounded_wait": (_c_int, [_c_int, _vp]),
@@ -168,8 +170,10 @@ def decode_workspace_bytes(B, Hq, Tk_max, d, chunk=256) -> int:
     return int(load_library().fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk))
 
 
-def decode_splitkv(q, k_cache, v_cache, seqlens, scale=None, chunk=256, workspace=None, out=None, lse=None):
-    """Split-KV decode.  q [B,Hq,d], caches [B,Tk_max,Hkv,d] bf16, seqlens int32 [B] (CUDA)."""
+def decode_splitkv(q, k_cache, v_cache, seqlens, scale=None, chunk=256, workspace=None, out=None, lse=None,
+                   window=None):
+    """Split-KV decode.  q [B,Hq,d], caches [B,Tk_max,Hkv,d] bf16, seqlens int32 [B] (CUDA).
+    ``window`` (int >= 1) keeps only the last `window` keys of each sequence."""
     lib = load_library()
     B, Hq, d = q.shape
     Tk_max, Hkv = k_cache.shape[1], k_cache.shape[2]
@@ -184,10 +188,14 @@ def decode_splitkv(q, k_cache, v_cache, seqlens, scale=None, chunk=256, workspac
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq), dtype=torch.float32, device=dev) if lse is None else lse
-    st = lib.fa_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse),
-                               _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tk_max, d, float(scale),
-                               int(chunk), _stream_ptr(dev))
-    _raise("fa_decode_splitkv", st)
+    args = (_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse), _ptr(workspace),
+            workspace.numel(), B, Hq, Hkv, Tk_max, d, float(scale), int(chunk))
+    if window is None:
+        st = lib.fa_decode_splitkv(*args, _stream_ptr(dev))
+        _raise("fa_decode_splitkv", st)
+    else:
+        st = lib.fa_decode_splitkv_window(*args, int(window), _stream_ptr(dev))
+        _raise("fa_decode_splitkv_window", st)
     return out, lse
 
 

@@ -441,11 +441,14 @@ size_t fa_decode_workspace_bytes(int B, int Hq, int Tk_max, int d, int chunk) {
   return round256((size_t)B * Hq * n * d * 4) + round256((size_t)B * Hq * n * 4);
 }
 
-int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
-                      void* o, float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv,
-                      int Tk_max, int d, float scale, int chunk, void* stream) {
+}  // extern "C"
+
+static int decode_impl(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k, void* o,
+                       float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tk_max, int d,
+                       float scale, int chunk, int window, void* stream) {
   if (B < 0 || Hq < 1 || Hkv < 1 || Tk_max < 0 || Hq % Hkv != 0 || !isfinite(scale))
     return FA_ERR_INVALID_ARG;
+  if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
@@ -478,6 +481,7 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, c
   p.lse = lse;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tk_max = Tk_max; p.chunk = chunk; p.nchunk = (int)n;
   p.n_items = (int)((size_t)B * Hkv * n);
+  p.window = window;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -511,6 +515,23 @@ int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, c
   else
     fa_decode_empty_kernel<128><<<blocks, 256, 0, s>>>(p);
   return launch_status();
+}
+
+extern "C" {
+
+int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
+                      void* o, float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv,
+                      int Tk_max, int d, float scale, int chunk, void* stream) {
+  return decode_impl(q, k_cache, v_cache, seqlens_k, o, lse, ws, ws_bytes, B, Hq, Hkv, Tk_max, d, scale, chunk, 0,
+                     stream);
+}
+
+int fa_decode_splitkv_window(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
+                             void* o, float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv,
+                             int Tk_max, int d, float scale, int chunk, int window, void* stream) {
+  if (window < 1) return FA_ERR_INVALID_ARG;
+  return decode_impl(q, k_cache, v_cache, seqlens_k, o, lse, ws, ws_bytes, B, Hq, Hkv, Tk_max, d, scale, chunk,
+                     window, stream);
 }
 
 int fa_check(void* stream) {

@@ -43,6 +43,7 @@ struct DecodeParams {
   float* lse;                // [B][Hq]
   int B, Hq, Hkv, Tk_max, chunk, nchunk;
   int n_items;               // B * Hkv * nchunk (items past a sequence's end are skipped)
+  int window;                // > 0: the query sees only the last `window` keys of its sequence
   float scale_log2;
   unsigned long long wait_limit_ns;
 };
@@ -150,7 +151,7 @@ fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
         const int b = bh / p.Hkv, hkv = bh % p.Hkv;
         const int k0 = c * p.chunk;
         const int seqlen = seqlen_of(b);
-        if (k0 >= seqlen) continue;
+        if (k0 >= seqlen || (p.window > 0 && k0 + p.chunk <= seqlen - p.window)) continue;
         const int nsub = (min(p.chunk, seqlen - k0) + C::SUB - 1) / C::SUB;
         // the G query rows of the group are contiguous: one bulk copy
         const int qs = qi & 1;
@@ -196,8 +197,10 @@ fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
     const int b = bh / p.Hkv, hkv = bh % p.Hkv;
     const int k0 = c * p.chunk;
     const int seqlen = seqlen_of(b);
-    if (k0 >= seqlen) continue;
+    if (k0 >= seqlen || (p.window > 0 && k0 + p.chunk <= seqlen - p.window)) continue;
     const int nkeys = min(p.chunk, seqlen - k0);
+    // keys of the chunk before this bound are outside the window
+    const int klo = p.window > 0 ? seqlen - p.window - k0 : -(1 << 30);
     const int nsub = (nkeys + C::SUB - 1) / C::SUB;
 
     // Q as the A operand (rows >= G are zero); scaling is applied to the
@@ -252,7 +255,8 @@ fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
       float sc[4] = {s0[0], s0[1], s1[0], s1[1]};
       const int kk[4] = {kb0, kb0 + 1, kb0 + 8, kb0 + 9};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sc[e] = (kk[e] < nkeys && real_row) ? sc[e] * p.scale_log2 : -INFINITY;
+      for (int e = 0; e < 4; ++e)
+        sc[e] = (kk[e] < nkeys && kk[e] >= klo && real_row) ? sc[e] * p.scale_log2 : -INFINITY;
       float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -351,22 +355,24 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const __grid_con
   const int seqlen = p.seqlens[b];
   const int nch = (seqlen + p.chunk - 1) / p.chunk;
   if (nch == 0) return;  // written by fa_decode_empty_kernel
+  // with a window the chunks before the first visible key were skipped
+  const int c_lo = p.window > 0 ? max(0, seqlen - p.window) / p.chunk : 0;
   constexpr int E = D / 32;
   const float* lse_c = p.ws_lse + (size_t)gw * p.nchunk;
   const float* o_c = p.ws_o + (size_t)gw * p.nchunk * D;
   float mx = -INFINITY;
-  for (int cc = lane; cc < nch; cc += 32) mx = fmaxf(mx, lse_c[cc]);
+  for (int cc = c_lo + lane; cc < nch; cc += 32) mx = fmaxf(mx, lse_c[cc]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   float sum = 0.f;
-  for (int cc = lane; cc < nch; cc += 32) sum += ex2_approx((lse_c[cc] - mx) * 1.4426950408889634f);
+  for (int cc = c_lo + lane; cc < nch; cc += 32) sum += ex2_approx((lse_c[cc] - mx) * 1.4426950408889634f);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
   const float lse = mx + logf(sum);
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  int cc = 0;
+  int cc = c_lo;
   for (; cc + 4 <= nch; cc += 4) {
     float wgt[4], vals[4][E];
 #pragma unroll

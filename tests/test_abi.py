@@ -111,3 +111,11 @@ def test_window_entry_points_reject_bad_window_on_host():
     assert lib.fa_forward_window(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 16, 16, 64, 1.0, 4, NULL) == 1
     assert lib.fa_forward_window(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 0, 16, 64, 1.0, 4, NULL) == 0
     assert lib.fa_forward_window(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 16, 16, 96, 1.0, 4, NULL) == 2
+
+
+def test_decode_window_rejects_bad_window_on_host():
+    lib = fa.load_library()
+    for w in (0, -1):
+        assert lib.fa_decode_splitkv_window(*([NULL] * 6), NULL, 0, 2, 32, 8, 1024, 128, 0.1, 256, w, NULL) == 1
+    # otherwise the same checks as fa_decode_splitkv (G = 16 unsupported)
+    assert lib.fa_decode_splitkv_window(*([NULL] * 6), NULL, 0, 2, 32, 2, 1024, 128, 0.1, 256, 8, NULL) == 2

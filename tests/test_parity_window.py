@@ -90,3 +90,23 @@ def test_window_long_sequence_sampled_rows():
         O, LSE = oracle.head_forward(q64[0, :, h], k64[0, :, h], v64[0, :, h], w.scale, True, rows=rows, window=W)
         assert_o_close(to_f64(o[0, rows, h]), O)
         assert_lse_close(lse[0, h, rows].numpy(), LSE)
+
+
+@pytest.mark.parametrize("Hq,Hkv,d,chunk,W,seqlens", [
+    (8, 2, 128, 256, 300, [1, 255, 256, 257, 1000]),   # window inside, across and beyond chunks
+    (4, 4, 64, 256, 1, [1, 64, 65, 777]),              # the last key only
+    (16, 2, 128, 512, 513, [3, 1000, 513, 514]),
+    (2, 2, 64, 64, 5000, [1, 63, 64, 65, 500]),        # wider than every sequence
+])
+def test_window_decode(Hq, Hkv, d, chunk, W, seqlens):
+    from workloads import decode_inputs
+    w = WORKLOADS[5].with_(Hq=Hq, Hkv=Hkv, d=d)
+    inp = decode_inputs(w, seed=77 + d + chunk + W, B=len(seqlens), Tk_max=1000, seqlens=seqlens)
+    dev = {n: t.cuda() for n, t in inp.items()}
+    o, lse = fa.decode_splitkv(dev["q"], dev["k_cache"], dev["v_cache"], dev["seqlens"], scale=w.scale,
+                               chunk=chunk, window=W)
+    assert fa.check() == 0
+    O, LSE = oracle.decode_forward(to_f64(inp["q"]), to_f64(inp["k_cache"]), to_f64(inp["v_cache"]),
+                                   inp["seqlens"].cpu().numpy(), w.scale, window=W)
+    assert_o_close(to_f64(o.cpu()), O)
+    assert_lse_close(lse.cpu().numpy(), LSE)

@@ -215,7 +215,7 @@ def oracle_heads(w, inp_cpu, heads, budget_s):
     return done, dt, done * per_head
 
 
-def oracle_decode(w, q, kc, vc, seqlens, budget_s):
+def oracle_decode(w, q, kc, vc, seqlens, budget_s, max_passes=None):
     """Run the oracle's decode (G query heads of one KV head at a time) over
     the given sequences; stop at the budget.  Returns (groups done, seconds,
     algorithmic bytes done: the K and V rows the query sees, q, o, lse)."""
@@ -223,7 +223,9 @@ def oracle_decode(w, q, kc, vc, seqlens, budget_s):
     from workloads import to_f64
     G = w.Hq // w.Hkv
     done, nbytes, t0 = 0, 0, time.perf_counter()
-    while True:   # passes over the given sequences until the budget is spent
+    passes = 0
+    while max_passes is None or passes < max_passes:   # passes until the budget is spent
+        passes += 1
         for b in range(q.shape[0]):
             L = int(seqlens[b])
             seen = min(L, w.window) if w.window else L
@@ -235,6 +237,7 @@ def oracle_decode(w, q, kc, vc, seqlens, budget_s):
                 nbytes += seen * w.d * 2 * 2 + G * (w.d * 2 * 2 + 4)
                 if time.perf_counter() - t0 >= budget_s:
                     return done, time.perf_counter() - t0, nbytes
+    return done, time.perf_counter() - t0, nbytes
 
 
 def cpu_baseline(w, inp_cpu, budget_s):
@@ -262,7 +265,7 @@ def run_reference_decode(args, w):
         b, hkv = groups[s % len(groups)]
         sub = w.with_(Hq=G, Hkv=1)
         return oracle_decode(sub, q[b:b + 1, hkv * G:(hkv + 1) * G], kc[b:b + 1, :, hkv:hkv + 1],
-                             vc[b:b + 1, :, hkv:hkv + 1], sl[b:b + 1], 1e9)
+                             vc[b:b + 1, :, hkv:hkv + 1], sl[b:b + 1], 1e9, max_passes=1)
 
     for s in range(args.warmup):
         one(s)

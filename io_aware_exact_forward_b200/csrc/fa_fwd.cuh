@@ -68,12 +68,17 @@ struct FwdCfg {
   static constexpr int OFF_RING = 4 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSTAGE * TILE_BYTES;
   // q_full[2], q_empty[2], kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2],
-  // p_full[2], o_final[2], mma_done
-  static constexpr int NBAR = 4 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+  // p_full[2], o_final[2], mma_done, s_free[2], p_free[2]
+  static constexpr int NBAR = 4 + 2 * NSTAGE + 2 + 2 + 2 + 1 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 320;
   static constexpr int TMEM_COLS = 512;
+  // d = 64: P gets its own tensor-memory columns (after S0, S1, O0, O1), so
+  // that the next S can be computed as soon as the softmax has loaded this
+  // one, overlapping the softmax; d = 128 has no room and writes P over S.
+  static constexpr bool SEP_P = (D == 64);
+  static constexpr int TM_P = 256 + 2 * D;       // P0, P1: 64 columns each (SEP_P)
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
   static constexpr float RESCALE_THRESHOLD = 8.0f;
@@ -135,6 +140,8 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
   auto bar_p_full = [&](int w) { return bar_base + 8u * (6 + 2 * C::NSTAGE + w); };
   auto bar_o_final = [&](int w) { return bar_base + 8u * (8 + 2 * C::NSTAGE + w); };
   const uint32_t bar_mma_done = bar_base + 8u * (10 + 2 * C::NSTAGE);
+  auto bar_s_free = [&](int w) { return bar_base + 8u * (11 + 2 * C::NSTAGE + w); };  // softmax loaded S
+  auto bar_p_free = [&](int w) { return bar_base + 8u * (13 + 2 * C::NSTAGE + w); };  // PV read P, wrote O
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   auto q_addr = [&](int qb, int w) { return sbase + C::OFF_Q + (2 * qb + w) * C::TILE_BYTES; };
@@ -158,6 +165,8 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
       mbar_init(bar_s_full(w), 1);
       mbar_init(bar_p_full(w), 128);
       mbar_init(bar_o_final(w), 1);
+      mbar_init(bar_s_free(w), 128);
+      mbar_init(bar_p_free(w), 1);
     }
     mbar_init(bar_mma_done, 1);
     fence_barrier_init();
@@ -235,52 +244,113 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
       };
       bool ok = true;
       int qi = 0, g = 0;  // items with work, global KV tile counter
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        const FwdItem it = fwd_item<D>(p, item);
-        if (it.n_kv == 0) continue;
-        const int qb = qi & 1;
-        ok = mbar_wait(bar_q_full(qb), (qi >> 1) & 1, wc);
-        if (!ok) break;
-        tc_fence_after();
-        int sV_prev = 0;
-        for (int j = 0; j < it.n_kv && ok; ++j) {
-          const int gt = g + j;
-          const int iK = 2 * gt, iV = 2 * gt + 1;
-          const int sK = iK % C::NSTAGE, sV = iV % C::NSTAGE;
-          ok = mbar_wait(bar_kv_full(sK), (iK / C::NSTAGE) & 1, wc);
+      if constexpr (C::SEP_P) {
+        // P lives in its own columns: for every KV tile j, S_0(j) and S_1(j)
+        // are issued as soon as the softmax warpgroups have loaded S(j-1)
+        // (s_free), and PV_w(j-1) once P_w(j-1) is written (p_full); each PV
+        // commits p_free, which releases the P columns and O to the softmax.
+        const uint32_t tP[2] = {tmem + C::TM_P, tmem + C::TM_P + 64};
+        auto issue_pv_p = [&](int w, int sV, bool first) {
+#pragma unroll
+          for (int k = 0; k < C::BN / 16; ++k) {
+            mma_ts(tO[w], tP[w] + k * 8, smem_desc_sw128(stage_addr(sV) + k * 16 * 128, C::BOX_BYTES, 1024),
+                   C::IDESC_O, (!first) || k > 0);
+          }
+        };
+        for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+          const FwdItem it = fwd_item<D>(p, item);
+          if (it.n_kv == 0) continue;
+          const int qb = qi & 1;
+          ok = mbar_wait(bar_q_full(qb), (qi >> 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          issue_s(0, q_addr(qb, 0), sK);
-          mma_commit(bar_s_full(0));
-          if (j > 0) {
-            ok = mbar_wait(bar_p_full(1), (gt - 1) & 1, wc);
+          for (int j = 0; j <= it.n_kv && ok; ++j) {
+            const int gt = g + j;
+            if (j < it.n_kv) {
+              const int iK = 2 * gt, sK = iK % C::NSTAGE;
+              ok = mbar_wait(bar_kv_full(sK), (iK / C::NSTAGE) & 1, wc);
+#pragma unroll
+              for (int w = 0; w < 2; ++w) {
+                if (ok && gt > 0) ok = mbar_wait(bar_s_free(w), (gt - 1) & 1, wc);
+                if (!ok) break;
+                tc_fence_after();
+                issue_s(w, q_addr(qb, w), sK);
+                mma_commit(bar_s_full(w));
+              }
+              if (!ok) break;
+              mma_commit(bar_kv_empty(sK));
+            }
+            if (j > 0) {
+              // PV of the previous tile
+              const int iV = 2 * (gt - 1) + 1, sV = iV % C::NSTAGE;
+              ok = mbar_wait(bar_kv_full(sV), (iV / C::NSTAGE) & 1, wc);
+              const bool last = j == it.n_kv;
+#pragma unroll
+              for (int w = 0; w < 2; ++w) {
+                if (ok) ok = mbar_wait(bar_p_full(w), (gt - 1) & 1, wc);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv_p(w, sV, j == 1);
+                mma_commit(bar_p_free(w));
+                if (last) mma_commit(bar_o_final(w));
+              }
+              if (!ok) break;
+              mma_commit(bar_kv_empty(sV));
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar_q_empty(qb));
+          g += it.n_kv;
+          ++qi;
+        }
+      } else {
+        for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+          const FwdItem it = fwd_item<D>(p, item);
+          if (it.n_kv == 0) continue;
+          const int qb = qi & 1;
+          ok = mbar_wait(bar_q_full(qb), (qi >> 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          int sV_prev = 0;
+          for (int j = 0; j < it.n_kv && ok; ++j) {
+            const int gt = g + j;
+            const int iK = 2 * gt, iV = 2 * gt + 1;
+            const int sK = iK % C::NSTAGE, sV = iV % C::NSTAGE;
+            ok = mbar_wait(bar_kv_full(sK), (iK / C::NSTAGE) & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(1, sV_prev, j - 1 == 0);
-            mma_commit(bar_kv_empty(sV_prev));
+            issue_s(0, q_addr(qb, 0), sK);
+            mma_commit(bar_s_full(0));
+            if (j > 0) {
+              ok = mbar_wait(bar_p_full(1), (gt - 1) & 1, wc);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(1, sV_prev, j - 1 == 0);
+              mma_commit(bar_kv_empty(sV_prev));
+            }
+            issue_s(1, q_addr(qb, 1), sK);
+            mma_commit(bar_s_full(1));
+            mma_commit(bar_kv_empty(sK));
+            ok = mbar_wait(bar_p_full(0), gt & 1, wc);
+            if (!ok) break;
+            ok = mbar_wait(bar_kv_full(sV), (iV / C::NSTAGE) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(0, sV, j == 0);
+            sV_prev = sV;
           }
-          issue_s(1, q_addr(qb, 1), sK);
-          mma_commit(bar_s_full(1));
-          mma_commit(bar_kv_empty(sK));
-          ok = mbar_wait(bar_p_full(0), gt & 1, wc);
           if (!ok) break;
-          ok = mbar_wait(bar_kv_full(sV), (iV / C::NSTAGE) & 1, wc);
+          mma_commit(bar_o_final(0));
+          ok = mbar_wait(bar_p_full(1), (g + it.n_kv - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(0, sV, j == 0);
-          sV_prev = sV;
+          issue_pv(1, sV_prev, it.n_kv - 1 == 0);
+          mma_commit(bar_kv_empty(sV_prev));
+          mma_commit(bar_o_final(1));
+          mma_commit(bar_q_empty(qb));
+          g += it.n_kv;
+          ++qi;
         }
-        if (!ok) break;
-        mma_commit(bar_o_final(0));
-        ok = mbar_wait(bar_p_full(1), (g + it.n_kv - 1) & 1, wc);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, sV_prev, it.n_kv - 1 == 0);
-        mma_commit(bar_kv_empty(sV_prev));
-        mma_commit(bar_o_final(1));
-        mma_commit(bar_q_empty(qb));
-        g += it.n_kv;
-        ++qi;
       }
       // Wait until every MMA issued above has completed before teardown.
       mma_commit(bar_mma_done);
@@ -293,6 +363,7 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + w * 128 + lane_off;
     const uint32_t tO = tmem + 256 + w * D + lane_off;
+    const uint32_t tP = tmem + C::TM_P + w * 64 + lane_off;  // P's own columns (SEP_P)
     bool ok = true;
     int qi = 0, g = 0;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -310,6 +381,11 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, su + c * 32);
         tmem_wait_ld();
+        if constexpr (C::SEP_P) {
+          // S is in registers: the next S may overwrite its columns
+          tc_fence_before();
+          mbar_arrive(bar_s_free(w));
+        }
         const int nvalid = key_limit - (it.kv0 + j) * C::BN;  // columns >= nvalid are masked
         const int nlo = key_lo - (it.kv0 + j) * C::BN;         // and columns < nlo
         const bool masked = __any_sync(0xffffffffu, nvalid < C::BN || nlo > 0);
@@ -357,12 +433,24 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
         }
         const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
         l += a.x + a.y;
-        tmem_st32(tS, su);
-        tmem_st32(tS + 32, su + 32);
+        if constexpr (C::SEP_P) {
+          // P's columns and O are free once the previous tile's PV completed
+          if (g + j > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_p_free(w), (g + j - 1) & 1, wc));
+            if (!ok) break;
+          }
+          tc_fence_after();
+          tmem_st32(tP, su);
+          tmem_st32(tP + 32, su + 32);
+        } else {
+          tmem_st32(tS, su);
+          tmem_st32(tS + 32, su + 32);
+        }
         if (j > 0 && __any_sync(0xffffffffu, move)) {
-          // O row *= alpha.  The PV of the previous tile has completed: the
-          // commit behind s_full tracks every MMA issued before it, and the
-          // PV of this tile waits for p_full below.
+          // O row *= alpha.  The PV of the previous tile has completed (with
+          // P over S, the commit behind s_full tracks every MMA issued before
+          // it; with P apart, p_free was awaited above), and the PV of this
+          // tile waits for p_full below.
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];

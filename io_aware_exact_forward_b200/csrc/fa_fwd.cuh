@@ -82,10 +82,12 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
   static constexpr float RESCALE_THRESHOLD = 8.0f;
-  // Pairs of S columns whose exponentials use exp2_poly2 (3 of every 8 at
-  // d = 128, where the shared MUFU unit limits the softmax; none at d = 64,
-  // where the extra FMA-pipe instructions cost more than they save).
-  static constexpr bool poly_pair(int c) { return D == 128 && ((c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6); }
+  // Pairs of S columns whose exponentials use exp2_poly2: 3 of every 8 at
+  // d = 128, where the shared MUFU unit limits the softmax, 1 of every 8 at
+  // d = 64 (more costs more FMA-pipe issue than it saves; measured).
+  static constexpr bool poly_pair(int c) {
+    return D == 128 ? ((c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6) : ((c & 7) == 3);
+  }
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
 };
 

@@ -78,6 +78,8 @@ struct FwdCfg {
   // that the next S can be computed as soon as the softmax has loaded this
   // one, overlapping the softmax; d = 128 has no room and writes P over S.
   static constexpr bool SEP_P = (D == 64);
+  // With SEP_P the ring holds (K_j, V_j) pairs with one barrier pair each.
+  static constexpr int NPAIR = NSTAGE / 2;
   static constexpr int TM_P = 256 + 2 * D;       // P0, P1: 64 columns each (SEP_P)
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
@@ -203,16 +205,31 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
           tma_load_4d(q_addr(qb, 1) + kb * C::BOX_BYTES, &p.tm_q, bar_q_full(qb), kb * 64, it.h, it.m0 + C::BM, it.b);
         }
         for (int j = 0; j < it.n_kv && ok; ++j) {
-          for (int which = 0; which < 2 && ok; ++which, ++idx) {
-            const int s = idx % C::NSTAGE;
-            const int round = idx / C::NSTAGE;
-            if (round > 0) ok = mbar_wait(bar_kv_empty(s), (round - 1) & 1, wc);
+          if constexpr (C::SEP_P) {
+            // K_j and V_j share one stage pair and one full/empty barrier
+            const int gp = idx >> 1, pi = gp % C::NPAIR, round = gp / C::NPAIR;
+            if (round > 0) ok = mbar_wait(bar_kv_empty(pi), (round - 1) & 1, wc);
             if (!ok) break;
-            mbar_arrive_expect_tx(bar_kv_full(s), C::TILE_BYTES);
-            const CUtensorMap* tm = which ? &p.tm_v : &p.tm_k;
-            for (int kb = 0; kb < C::NBOX; ++kb)
-              tma_load_4d(stage_addr(s) + kb * C::BOX_BYTES, tm, bar_kv_full(s), kb * 64, it.hkv,
+            mbar_arrive_expect_tx(bar_kv_full(pi), 2 * C::TILE_BYTES);
+            for (int kb = 0; kb < C::NBOX; ++kb) {
+              tma_load_4d(stage_addr(2 * pi) + kb * C::BOX_BYTES, &p.tm_k, bar_kv_full(pi), kb * 64, it.hkv,
                           (it.kv0 + j) * C::BN, it.b);
+              tma_load_4d(stage_addr(2 * pi + 1) + kb * C::BOX_BYTES, &p.tm_v, bar_kv_full(pi), kb * 64, it.hkv,
+                          (it.kv0 + j) * C::BN, it.b);
+            }
+            idx += 2;
+          } else {
+            for (int which = 0; which < 2 && ok; ++which, ++idx) {
+              const int s = idx % C::NSTAGE;
+              const int round = idx / C::NSTAGE;
+              if (round > 0) ok = mbar_wait(bar_kv_empty(s), (round - 1) & 1, wc);
+              if (!ok) break;
+              mbar_arrive_expect_tx(bar_kv_full(s), C::TILE_BYTES);
+              const CUtensorMap* tm = which ? &p.tm_v : &p.tm_k;
+              for (int kb = 0; kb < C::NBOX; ++kb)
+                tma_load_4d(stage_addr(s) + kb * C::BOX_BYTES, tm, bar_kv_full(s), kb * 64, it.hkv,
+                            (it.kv0 + j) * C::BN, it.b);
+            }
           }
         }
         ++qi;
@@ -220,8 +237,13 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
       if (!ok) {
         // Let every copy already issued land before the CTA can exit.
         for (int q = max(0, qi - 1); q <= qi; ++q) mbar_wait_drain(bar_q_full(q & 1), (q >> 1) & 1, p.wait_limit_ns);
-        for (int k = max(0, idx - C::NSTAGE); k < idx; ++k)
-          mbar_wait_drain(bar_kv_full(k % C::NSTAGE), (k / C::NSTAGE) & 1, p.wait_limit_ns);
+        if constexpr (C::SEP_P) {
+          for (int k = max(0, (idx >> 1) - C::NPAIR); k < (idx >> 1); ++k)
+            mbar_wait_drain(bar_kv_full(k % C::NPAIR), (k / C::NPAIR) & 1, p.wait_limit_ns);
+        } else {
+          for (int k = max(0, idx - C::NSTAGE); k < idx; ++k)
+            mbar_wait_drain(bar_kv_full(k % C::NSTAGE), (k / C::NSTAGE) & 1, p.wait_limit_ns);
+        }
       }
     }
   } else if (warp == 8) {
@@ -269,23 +291,21 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
           for (int j = 0; j <= it.n_kv && ok; ++j) {
             const int gt = g + j;
             if (j < it.n_kv) {
-              const int iK = 2 * gt, sK = iK % C::NSTAGE;
-              ok = mbar_wait(bar_kv_full(sK), (iK / C::NSTAGE) & 1, wc);
+              const int pi = gt % C::NPAIR;
+              ok = mbar_wait(bar_kv_full(pi), (gt / C::NPAIR) & 1, wc);  // K_j and V_j
 #pragma unroll
               for (int w = 0; w < 2; ++w) {
                 if (ok && gt > 0) ok = mbar_wait(bar_s_free(w), (gt - 1) & 1, wc);
                 if (!ok) break;
                 tc_fence_after();
-                issue_s(w, q_addr(qb, w), sK);
+                issue_s(w, q_addr(qb, w), 2 * pi);
                 mma_commit(bar_s_full(w));
               }
               if (!ok) break;
-              mma_commit(bar_kv_empty(sK));
             }
             if (j > 0) {
-              // PV of the previous tile
-              const int iV = 2 * (gt - 1) + 1, sV = iV % C::NSTAGE;
-              ok = mbar_wait(bar_kv_full(sV), (iV / C::NSTAGE) & 1, wc);
+              // PV of the previous tile (its V arrived with its K)
+              const int pi = (gt - 1) % C::NPAIR, sV = 2 * pi + 1;
               const bool last = j == it.n_kv;
 #pragma unroll
               for (int w = 0; w < 2; ++w) {
@@ -297,7 +317,7 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
                 if (last) mma_commit(bar_o_final(w));
               }
               if (!ok) break;
-              mma_commit(bar_kv_empty(sV));
+              mma_commit(bar_kv_empty(pi));
             }
           }
           if (!ok) break;

@@ -361,10 +361,17 @@ static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO
   const bool persistent = d == 64 && !causal;
   dim3 grid(persistent ? std::min(p.n_items, nsm) : p.n_items);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    fa_bwd_dkdv_kernel<64><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
-  else
-    fa_bwd_dkdv_kernel<128><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+  if (d == 64) {
+    if (window > 0)
+      fa_bwd_dkdv_kernel<64, true><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+    else
+      fa_bwd_dkdv_kernel<64, false><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+  } else {
+    if (window > 0)
+      fa_bwd_dkdv_kernel<128, true><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+    else
+      fa_bwd_dkdv_kernel<128, false><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+  }
   return launch_status();
 }
 

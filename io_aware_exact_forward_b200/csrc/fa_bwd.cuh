@@ -241,7 +241,9 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   return it;
 }
 
-template <int D>
+// WIN: sliding-window masking compiled in (a separate instantiation, so
+// that the plain path keeps its registers).
+template <int D, bool WIN>
 __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -526,8 +528,8 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         const float* lrow = lse_s + s * 128 + 64 * half;
         const int cmin = p.causal ? qmin - q0 - 64 * half : 0;  // columns < cmin are masked
         // and, with a window, columns >= cmax (queries past this key's window)
-        const int cmax = p.window > 0 ? qmin + p.window - q0 - 64 * half : (1 << 30);
-        const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > 0 || cmax < 64);
+        const int cmax = WIN ? qmin + p.window - q0 - 64 * half : (1 << 30);
+        const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > 0 || (WIN && cmax < 64));
         // 64 query columns in four 16-column chunks; the load of chunk c+1
         // overlaps the exponentials of chunk c.  P^T (bf16 pairs) goes to
         // the first 32 columns of this warp's 64, never ahead of its loads.
@@ -548,8 +550,8 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             float p0 = ex2_approx(x.x);
             float p1 = ex2_approx(x.y);
             if (masked) {
-              if (!key_ok || col < cmin || col >= cmax) p0 = 0.f;
-              if (!key_ok || col + 1 < cmin || col + 1 >= cmax) p1 = 0.f;
+              if (!key_ok || col < cmin || (WIN && col >= cmax)) p0 = 0.f;
+              if (!key_ok || col + 1 < cmin || (WIN && col + 1 >= cmax)) p1 = 0.f;
             }
             pk[e] = pack_bf16x2(p0, p1);
           }
@@ -650,21 +652,23 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             const float2 r = __fmul2_rn(pf, t);
             pp[8 * c + e] = pack_bf16x2(r.x, r.y);
           }
-        }
-        if (gi > 0) {
-          // The shared dS tile is still an operand of the previous tile's
-          // dK and dQ MMAs until they complete (this tile's dP^T can
-          // complete before them); the arithmetic above overlaps that wait.
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
-          if (!ok) break;
-        }
-        // dS into shared memory: row j of box `half`, eight 16-byte chunks,
-        // 128-byte swizzle (chunk ^ (row % 8)).
+          if (c == 0 && gi > 0) {
+            // The shared dS tile is still an operand of the previous tile's
+            // dK and dQ MMAs until they complete (this tile's dP^T can
+            // complete before them).
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
+            if (!ok) break;
+          }
+          // dS into shared memory: row j of box `half`, 16-byte chunks 2c and
+          // 2c+1, 128-byte swizzle (chunk ^ (row % 8)).
 #pragma unroll
-        for (int chunk = 0; chunk < 8; ++chunk)
-          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (j & 7)) << 4)) =
-              make_uint4(pp[4 * chunk], pp[4 * chunk + 1], pp[4 * chunk + 2], pp[4 * chunk + 3]);
+          for (int q = 0; q < 2; ++q) {
+            const int chunk = 2 * c + q;
+            *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (j & 7)) << 4)) =
+                make_uint4(pp[8 * c + 4 * q], pp[8 * c + 4 * q + 1], pp[8 * c + 4 * q + 2], pp[8 * c + 4 * q + 3]);
+          }
+        }
         if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_before();
@@ -750,12 +754,15 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
 }
 
 static int bwd_setup() {
-  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64>),
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<64>::SMEM_BYTES) != cudaSuccess)
-    return FA_ERR_CUDA;
-  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128>),
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<128>::SMEM_BYTES) != cudaSuccess)
-    return FA_ERR_CUDA;
+  const void* kernels[4] = {reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, true>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, true>)};
+  const int bytes[4] = {BwdCfg<64>::SMEM_BYTES, BwdCfg<64>::SMEM_BYTES, BwdCfg<128>::SMEM_BYTES,
+                        BwdCfg<128>::SMEM_BYTES};
+  for (int i = 0; i < 4; ++i)
+    if (cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes[i]) != cudaSuccess)
+      return FA_ERR_CUDA;
   return FA_OK;
 }
 

@@ -9,23 +9,27 @@
 //   preprocess   D_i = sum_c dO_ic O_ic (fp32), LSE in log2 units (+inf for a
 //                row that saw no key, so that its P is exactly 0), dQ
 //                accumulator zeroed.                          (memory-bound)
-//   dkdv         one CTA per (128-key tile, KV head, batch).  K and V stay in
-//                shared memory; the CTA walks the query tiles of every query
-//                head of its GQA group.  Per tile, in tensor memory:
-//                  S^T = K Q^T, dP^T = V dO^T          (SS MMAs)
+//   dkdv         one work item per (128-key tile, KV head, batch).  K and V
+//                stay in shared memory; the item walks the query tiles of
+//                every query head of its GQA group.  Per tile:
+//                  S^T = K Q^T, dP^T = V dO^T          (SS MMAs, TMEM)
 //                  P^T = 2^{S^T*scale*log2e - LSE2}   (P warps, bf16 into
-//                        half of the S^T columns)
-//                  dV += P^T dO                         (TS MMA)
-//                  dS^T = P^T * (dP^T - D)             (dS warps, bf16 into
-//                        the other half of the S^T columns, and dS into
-//                        shared memory as an A operand)
-//                  dK += dS^T Q                         (TS MMA)
-//                  dQ_tile = dS K                       (SS MMA)
+//                        the S^T columns)
+//                  dV += P^T dO                         (TS MMA, P^T from TMEM)
+//                  dS = P^T * (dP^T - D)               (dS warps, bf16 into
+//                        a swizzled shared-memory tile: key rows, query
+//                        columns)
+//                  dK += dS^T Q                         (SS MMA, the tile
+//                        read K-major)
+//                  dQ_tile = dS K                       (SS MMA, the tile
+//                        read MN-major)
 //                At d = 64 (two S^T buffers) the next tile's S^T is issued
 //                ahead and its dP^T as soon as the dS warps have read this
-//                tile's; at d = 128 (one S^T buffer) dQ_tile lands in the dP^T
-//                columns, so that the next S^T follows dQ at once and the
-//                next dP^T follows the dQ read-out.
+//                tile's; at d = 128 (one S^T buffer) the next S^T follows dV
+//                once the dS warps hold this tile's P^T in registers, and
+//                dQ_tile lands in the dP^T columns, so the next dP^T follows
+//                the dQ read-out.  A sliding window is a separate
+//                instantiation (its masking costs registers).
 //                dQ_tile is read by a second warpgroup, staged in shared
 //                memory and added into an fp32 accumulator in global memory
 //                with bulk tensor reduce-adds (every KV tile contributes to
@@ -33,10 +37,10 @@
 //                group's heads in tensor memory, so the GQA sum needs no
 //                atomics.
 //   dq_convert   dq = bf16(accumulator).
-// Warp roles in dkdv: 0-7 P^T and 8-15 dS (two warps per TMEM lane quarter,
-// one per half of the 128 query columns, so that one warp computes while the
-// other waits for its tensor-memory loads), 16-19 dQ reduction (one query
-// row per thread), 20 MMA issuer, 21 TMA producer.
+// Warp roles in dkdv: 0-7 P^T and, at an item's end, dK/dV out; 8-15 dS
+// (two warps per TMEM lane quarter, one per half of the 128 query columns);
+// 16-19 dQ read-out and reduce-adds (one query row per thread); 20 MMA
+// issuer; 21 TMA producer.
 #pragma once
 
 #include "fa_ptx.cuh"

@@ -697,45 +697,51 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         // The four warps meet at named barriers below: after an expired wait
         // they still pass them, and all stop together at the end.
         if (ok) tc_fence_after();
+        // Passes of BPP 32-column boxes: TMEM loads, then staging and bulk
+        // reduce-adds; the columns are released after the last pass's
+        // loads.  d = 64 takes one box per pass (fewer live registers, no
+        // spills); d = 128 two, which releases its four boxes sooner.
+        constexpr int BPP = (D == 64) ? 1 : 2;
 #pragma unroll
-        for (int pr = 0; pr < D / 64; ++pr) {
-          // 64 columns (two fp32 boxes) per pass; the tensor-memory columns
-          // are released after the last pass's loads.
-          uint32_t v[2][32];
+        for (int pr = 0; pr < D / 32 / BPP; ++pr) {
+          uint32_t v[BPP][32];
           if (ok) {
-            tmem_ld32(tDQ + 64 * pr, v[0]);
-            tmem_ld32(tDQ + 64 * pr + 32, v[1]);
+#pragma unroll
+            for (int b = 0; b < BPP; ++b) tmem_ld32(tDQ + 32 * (pr * BPP + b), v[b]);
             tmem_wait_ld();
-            if (pr + 1 == D / 64) {
+            if (pr + 1 == D / 32 / BPP) {
               tc_fence_before();
               mbar_arrive(bar_dq_free(buf));
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[0][i] = v[1][i] = 0u;  // a stopped warp adds nothing
+            for (int b = 0; b < BPP; ++b)
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[b][i] = 0u;  // a stopped warp adds nothing
           }
 #pragma unroll
-          for (int box = 0; box < 2; ++box) {
+          for (int b = 0; b < BPP; ++b) {
+            const int bx = pr * BPP + b;
             // Before a staging box is refilled, the bulk reduce that last
             // read it must have finished reading.
-            const uint32_t slot = C::OFF_DQS + (box % C::NDQS) * C::BOX_BYTES;
-            if (box == 0 || C::NDQS == 1) {
+            const uint32_t slot = C::OFF_DQS + (bx % C::NDQS) * C::BOX_BYTES;
+            if (bx % C::NDQS == 0) {
               if (threadIdx.x == lead) bulk_wait_group_read0();
               named_bar_sync(2, 128);
             }
 #pragma unroll
             for (int chunk = 0; chunk < 8; ++chunk) {
               *reinterpret_cast<float4*>(smem + slot + r * 128 + ((chunk ^ (r & 7)) << 4)) =
-                  make_float4(__uint_as_float(v[box][4 * chunk]) * p.scale,
-                              __uint_as_float(v[box][4 * chunk + 1]) * p.scale,
-                              __uint_as_float(v[box][4 * chunk + 2]) * p.scale,
-                              __uint_as_float(v[box][4 * chunk + 3]) * p.scale);
+                  make_float4(__uint_as_float(v[b][4 * chunk]) * p.scale,
+                              __uint_as_float(v[b][4 * chunk + 1]) * p.scale,
+                              __uint_as_float(v[b][4 * chunk + 2]) * p.scale,
+                              __uint_as_float(v[b][4 * chunk + 3]) * p.scale);
             }
             fence_proxy_async_smem();
-            if (pr + 1 == D / 64 && box == 1 && threadIdx.x == lead) *stop_flag = *abort_flag;
+            if (bx + 1 == D / 32 && threadIdx.x == lead) *stop_flag = *abort_flag;
             named_bar_sync(2, 128);
             if (threadIdx.x == lead && !*stop_flag) {
-              tma_reduce_add_4d(&p.tm_dq, sbase + slot, (2 * pr + box) * 32, h, q0, I.b);
+              tma_reduce_add_4d(&p.tm_dq, sbase + slot, bx * 32, h, q0, I.b);
               bulk_commit_group();
             }
           }

@@ -62,6 +62,7 @@ __all__ = [
     "decode_forward",
     "online_softmax_row",
     "combine_partials",
+    "merge_partials",
     "brute_force_row",
 ]
 
@@ -283,6 +284,24 @@ def combine_partials(o_parts, lse_parts):
     w = np.exp(lse_parts - m)
     lse = m + math.log(w.sum())
     return (np.exp(lse_parts - lse)[:, None] * o_parts).sum(axis=0), lse
+
+
+def merge_partials(o_parts, lse_parts):
+    """Row-wise combine of R partial results of the same rows, e.g. decodes
+    of R disjoint shares of every sequence's keys on R devices (FlashDecoding's
+    split [FA §"In practice"] across devices).  o_parts [R, ..., d],
+    lse_parts [R, ...]; each row is merged by ``combine_partials``.  Returns
+    O [..., d], LSE [...]."""
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    R = lse_parts.shape[0]
+    rows = lse_parts.reshape(R, -1)
+    orows = o_parts.reshape(R, rows.shape[1], o_parts.shape[-1])
+    O = np.zeros(orows.shape[1:])
+    LSE = np.empty(rows.shape[1])
+    for i in range(rows.shape[1]):
+        O[i], LSE[i] = combine_partials(orows[:, i], rows[:, i])
+    return O.reshape(o_parts.shape[1:]), LSE.reshape(lse_parts.shape[1:])
 
 
 def brute_force_row(scores, values):

@@ -336,6 +336,58 @@ def test_decode_is_prefill_row_over_prefix():
     np.testing.assert_allclose(O[0], np.repeat(vc[0, 0], Hq // Hkv, axis=0), rtol=1e-15)
 
 
+def test_merge_of_key_shares_is_full_decode():
+    """Decoding disjoint shares of every sequence's keys (any split, empty
+    shares included) and merging the shares' (O, LSE) by log-sum-exp gives
+    the decode over all keys: the softmax over a union of key sets."""
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, d, Tmax, R = 3, 4, 2, 5, 50, 3
+    q = rng.standard_normal((B, Hq, d))
+    kc, vc = rng.standard_normal((B, Tmax, Hkv, d)), rng.standard_normal((B, Tmax, Hkv, d))
+    seqlens = [1, 23, 50]
+    O_ref, L_ref = oracle.decode_forward(q, kc, vc, seqlens, 0.4)
+    for contiguous in (True, False):
+        shares = [[] for _ in range(R)]
+        for b, n in enumerate(seqlens):
+            pos = np.arange(n) if contiguous else rng.permutation(n)
+            cuts = sorted(rng.integers(0, n + 1, size=R - 1)) if not contiguous else [n // 3, 2 * n // 3]
+            for r, part in enumerate(np.split(pos, cuts)):
+                shares[r].append(part)
+        o_parts, l_parts = [], []
+        for r in range(R):
+            ks, vs = np.zeros_like(kc), np.zeros_like(vc)
+            sl = []
+            for b in range(B):
+                idx = shares[r][b]
+                ks[b, :len(idx)], vs[b, :len(idx)] = kc[b, idx], vc[b, idx]
+                sl.append(len(idx))
+            o, l = oracle.decode_forward(q, ks, vs, sl, 0.4)
+            o_parts.append(o)
+            l_parts.append(l)
+        assert any(len(shares[r][0]) == 0 for r in range(R))   # sequence 0 has empty shares
+        O, L = oracle.merge_partials(np.stack(o_parts), np.stack(l_parts))
+        np.testing.assert_allclose(O, O_ref, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(L, L_ref, rtol=1e-13)
+
+
+def test_merge_closed_forms():
+    # weights e^{LSE_r}: LSE = (0, ln 3) puts 1/4 and 3/4 on the two partials
+    O, L = oracle.merge_partials(np.array([[[1.0, 0.0]], [[0.0, 1.0]]]), np.array([[0.0], [math.log(3.0)]]))
+    np.testing.assert_allclose(O[0], [0.25, 0.75], rtol=1e-15)
+    assert math.isclose(L[0], math.log(4.0), rel_tol=1e-15)
+    # two equal partials: the same output, LSE + ln 2
+    o = np.array([[0.3, -1.2, 4.0]])
+    O, L = oracle.merge_partials(np.stack([o, o]), np.array([[1.7], [1.7]]))
+    np.testing.assert_allclose(O, o, rtol=1e-15)
+    assert math.isclose(L[0], 1.7 + math.log(2.0), rel_tol=1e-15)
+    # a partial that saw no key (LSE = -inf) changes nothing; all of them empty gives 0, -inf
+    O, L = oracle.merge_partials(np.stack([o, np.zeros_like(o)]), np.array([[0.5], [-np.inf]]))
+    np.testing.assert_allclose(O, o, rtol=1e-15)
+    assert L[0] == 0.5
+    O, L = oracle.merge_partials(np.zeros((3, 1, 3)), np.full((3, 1), -np.inf))
+    assert (O == 0).all() and L[0] == -np.inf
+
+
 def test_row_panels_do_not_change_results():
     """Rows are processed in panels; a long causal head must equal the
     brute-force row for rows in different panels."""

@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--window", type=int, default=None,
                     help="sliding window of that many keys (prefill: implies causal; decode: last keys)")
+    ap.add_argument("--cp", action="store_true",
+                    help="decode only: context-parallel, every sequence's cache cut into one share per GPU")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (smaller cases for profiler captures only)")
     return ap.parse_args()
@@ -678,6 +680,132 @@ def run_decode(args, w, rank, world, dist):
     return 0
 
 
+def run_decode_cp(args, w, rank, world, dist):
+    """Context-parallel decode of the same batch: every sequence's cache is
+    cut into `world` contiguous shares and rank r holds share r.  One step is
+    fa_decode_splitkv_partial on the local share, one NCCL all-gather of the
+    packed fp32 (O, LSE) blocks and fa_decode_merge.  The whole batch's
+    algorithmic bytes are fixed as N grows (strong scaling); value is those
+    bytes per step over the slowest rank's step time."""
+    import ctypes
+    import torch
+    import io_aware_exact_forward_b200 as fa
+    from io_aware_exact_forward_b200 import context_parallel as cp
+    from workloads import decode_inputs
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    lib = fa.load_library()
+    full = decode_inputs(w, device=dev)            # the same batch on every rank
+    B, Hq, Hkv, Tk_max, d, chunk = w.B, w.Hq, w.Hkv, w.T, w.d, w.chunk
+    shard_len = (Tk_max + world - 1) // world
+    lo = rank * shard_len
+    q, sl_full = full["q"], full["seqlens"]
+    kc = full["k_cache"][:, lo:lo + shard_len].contiguous()
+    vc = full["v_cache"][:, lo:lo + shard_len].contiguous()
+    del full
+    torch.cuda.empty_cache()
+    sl = cp.shard_seqlens(sl_full, rank, shard_len)
+    Tk_loc = kc.shape[1]
+    total_keys = int(sl_full.sum().item())
+    n = cp.packed_block_floats(B, Hq, d)
+    n_o = B * Hq * d
+    block = torch.empty(n, dtype=torch.float32, device=dev)
+    gathered = torch.empty(world * n, dtype=torch.float32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    wsb = lib.fa_decode_workspace_bytes(B, Hq, Tk_loc, d, chunk)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    P = ctypes.c_void_p
+    stream = torch.cuda.current_stream(dev)
+    sp = P(stream.cuda_stream)
+    part_args = (P(q.data_ptr()), P(kc.data_ptr()), P(vc.data_ptr()), P(sl.data_ptr()), P(block.data_ptr()),
+                 P(block.data_ptr() + 4 * n_o), P(ws.data_ptr()), wsb, B, Hq, Hkv, Tk_loc, d, w.scale, chunk, sp)
+    merge_args = (P(gathered.data_ptr()), n, P(gathered.data_ptr() + 4 * n_o), n, P(o.data_ptr()),
+                  P(lse.data_ptr()), world, B, Hq, d, sp)
+
+    def step():
+        st = lib.fa_decode_splitkv_partial(*part_args)
+        if st != 0:
+            raise RuntimeError(f"fa_decode_splitkv_partial: {fa.STATUS.get(st, st)}")
+        dist.all_gather_into_tensor(gathered, block)
+        st = lib.fa_decode_merge(*merge_args)
+        if st != 0:
+            raise RuntimeError(f"fa_decode_merge: {fa.STATUS.get(st, st)}")
+
+    alg_bytes = total_keys * Hkv * d * 2 * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
+
+    def barrier():
+        dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        barrier()
+    if lib.fa_check(sp) != 0:
+        raise RuntimeError("device status set during the timed region")
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    value = alg_bytes * args.steps / (ms * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            oo, ll = fa.decode_splitkv_cp(q, kc, vc, sl, scale=w.scale, chunk=chunk, workspace=ws)
+            ho.copy_(oo, non_blocking=True)
+            hlse.copy_(ll, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        f1.record(stream)
+        barrier()
+        e_ms = max_over_ranks(f0.elapsed_time(f1), dist, dev)
+        e2e = {"value": alg_bytes * args.e2e_steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hlse.numel() * hlse.element_size(),
+               "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps,
+               "note": "each rank's share of the KV cache and the sequence lengths stay resident"}
+    peaks = load_peaks()
+    if rank == 0:
+        line = {
+            "metric": "split-KV decode HBM GB/s (bf16 KV cache, 1xB200) and % of HBM peak",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "context_parallel": True, "B": B, "Hq": Hq, "Hkv": Hkv,
+                       "Tk_max": Tk_max, "shard_len": shard_len, "d": d, "chunk": chunk,
+                       "total_cached_tokens": total_keys, "l2": "KV cache larger than L2", "seed": w.seed},
+            "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_combine_kernel + fa_decode_merge_kernel",
+                         "bound": "hbm", "achieved": value / world, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": value / world / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy",
+                         "traffic": None, "algorithmic_per_launch": alg_bytes / world},
+            "gpu_launches": 4 * args.steps,   # split, combine, empty-sequence and merge kernels (plus NCCL's)
+            "clocks": clocks.summary(),
+            "cpu_baseline": None,
+            "e2e": e2e,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     from workloads import WORKLOADS
@@ -694,14 +822,22 @@ def main():
     dist = None
     if args.impl == "reference":
         return run_reference(args, w, rank)
-    if world > 1:
+    if args.cp and (not w.decode or w.window):
+        print("--cp applies to the decode workload without a window", file=sys.stderr)
+        return 2
+    if world > 1 or args.cp:
         import datetime
         import torch
         import torch.distributed as tdist
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29533")
+        tdist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
         dist = tdist
     try:
+        if w.decode and args.cp:
+            return run_decode_cp(args, w, rank, world, dist)
         if w.decode:
             return run_decode(args, w, rank, world, dist)
         return run_fa(args, w, rank, world, dist)

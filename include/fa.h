@@ -225,6 +225,54 @@ int fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_
                               void* stream);
 
 /*
+ * Context-parallel decode: one sequence's KV cache spread over several GPUs.
+ * Each GPU decodes its own share of the keys with fa_decode_splitkv_partial,
+ * the GPUs exchange their (O_r, LSE_r) rows (an all-gather, the caller's
+ * collective), and fa_decode_merge combines them.  This is FlashDecoding's
+ * split of the KV cache ("FlashAttention", interview track, section "In
+ * practice") taken across devices: the merge is the chunk merge of
+ * fa_decode_splitkv with devices in place of chunks,
+ *   LSE = log sum_r e^{LSE_r},  O = sum_r e^{LSE_r - LSE} O_r.
+ * Keys may be shared out in any way (the unmasked softmax does not depend on
+ * key order); no window is offered because the window of the full sequence is
+ * not a window of each share.
+ *
+ * fa_decode_splitkv_partial -- fa_decode_splitkv over this GPU's share, with
+ * the normalised output written in fp32 so that the merge does not round
+ * twice.
+ *   o     fp32 [B][Hq][d], 16-byte aligned;  lse fp32 [B][Hq].
+ *   A sequence whose share is empty (seqlens_k[b] == 0) gets O = 0 and
+ *   LSE = -inf, which the merge ignores.  Everything else (arguments,
+ *   workspace, errors, asynchrony) as fa_decode_splitkv.
+ */
+int fa_decode_splitkv_partial(const void* q, const void* k_cache, const void* v_cache,
+                              const int* seqlens_k, float* o, float* lse, void* ws, size_t ws_bytes,
+                              int B, int Hq, int Hkv, int Tk_max, int d, float scale, int chunk,
+                              void* stream);
+
+/*
+ * fa_decode_merge -- combines R partial decodes of the same B x Hq rows.
+ *   o_parts     device fp32; partial r is the [B][Hq][d] block starting at
+ *               o_parts + r * o_stride.  16-byte aligned.
+ *   o_stride    floats between consecutive O blocks: a multiple of 4 and,
+ *               when R > 1, at least B * Hq * d.
+ *   lse_parts   device fp32; partial r is the [B][Hq] block starting at
+ *               lse_parts + r * lse_stride.  4-byte aligned.
+ *   lse_stride  floats between consecutive LSE blocks; when R > 1, at least
+ *               B * Hq.  (O and LSE of one partial may share one packed
+ *               block: O first, LSE after it, both strides the block size.)
+ *   o           device bf16 [B][Hq][d] (16-byte aligned); lse device fp32 [B][Hq].
+ *   R           number of partials, 1 .. 2^20.   d in {64, 128}.
+ * A row with LSE_r = -inf in every partial gets O = 0 and LSE = -inf.
+ * Errors: FA_ERR_INVALID_ARG (sizes, null pointers, short stride),
+ * FA_ERR_UNSUPPORTED (d), FA_ERR_ALIGNMENT, FA_ERR_CUDA (launch), all before
+ * or at launch; B == 0 is a no-op.  Asynchronous on `stream`; nothing is
+ * allocated and the inputs are not modified.
+ */
+int fa_decode_merge(const float* o_parts, size_t o_stride, const float* lse_parts, size_t lse_stride,
+                    void* o, float* lse, int R, int B, int Hq, int d, void* stream);
+
+/*
  * fa_check -- synchronise `stream`, then read and clear the device status
  * word that kernels set when a bounded wait expires.  Returns FA_OK,
  * FA_ERR_TIMEOUT, or FA_ERR_CUDA if the synchronisation itself failed.

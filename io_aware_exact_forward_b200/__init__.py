@@ -12,10 +12,13 @@ from ._binding import (  # noqa: F401
     backward,
     backward_workspace_bytes,
     check,
+    decode_merge,
     decode_splitkv,
     decode_splitkv_noalloc,
+    decode_splitkv_partial,
     decode_workspace_bytes,
     forward,
     load_library,
     selftest_bounded_wait,
 )
+from .context_parallel import decode_splitkv_cp  # noqa: F401,E402

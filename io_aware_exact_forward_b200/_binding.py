@@ -45,6 +45,8 @@ SIGNATURES = {
     "fa_decode_splitkv_window": (_c_int, [_vp] * 6 + [_vp, _c_size] + [_c_int] * 5 + [_c_float, _c_int, _c_int,
                                                                                     _vp]),
     "fa_decode_splitkv_noalloc": (_c_int, [_vp] * 6 + [_c_int] * 5 + [_c_float, _c_int, _vp]),
+    "fa_decode_splitkv_partial": (_c_int, [_vp] * 6 + [_vp, _c_size] + [_c_int] * 5 + [_c_float, _c_int, _vp]),
+    "fa_decode_merge": (_c_int, [_vp, _c_size, _vp, _c_size, _vp, _vp] + [_c_int] * 4 + [_vp]),
     "fa_check": (_c_int, [_vp]),
     "fa_selftest_bounded_wait": (_c_int, [_c_int, _vp]),
     "fa_selftest_exp2_poly": (_c_int, [_vp, _vp, _c_int, _vp]),
@@ -217,6 +219,62 @@ def decode_splitkv_noalloc(q, k_cache, v_cache, seqlens, scale=None, chunk=256, 
     st = lib.fa_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse),
                                        B, Hq, Hkv, Tk_max, d, float(scale), int(chunk), _stream_ptr(dev))
     _raise("fa_decode_splitkv_noalloc", st)
+    return out, lse
+
+
+def decode_splitkv_partial(q, k_cache, v_cache, seqlens, scale=None, chunk=256, workspace=None, out=None,
+                           lse=None):
+    """Split-KV decode of this device's share of the keys with O kept in
+    fp32 (fa_decode_splitkv_partial), for a later decode_merge.  Shapes as in
+    decode_splitkv; ``out`` is float32 [B,Hq,d] and may be a view into a
+    larger packed buffer."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    Tk_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+    dev = q.device
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_dev(n, t, torch.bfloat16, dev)
+    _check_dev("seqlens", seqlens, torch.int32, dev)
+    if scale is None:
+        scale = d ** -0.5
+    need = decode_workspace_bytes(B, Hq, Tk_max, d, chunk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_dev("out", out, torch.float32, dev)
+    _check_dev("lse", lse, torch.float32, dev)
+    st = lib.fa_decode_splitkv_partial(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse),
+                                       _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tk_max, d, float(scale),
+                                       int(chunk), _stream_ptr(dev))
+    _raise("fa_decode_splitkv_partial", st)
+    return out, lse
+
+
+def decode_merge(o_parts, lse_parts, out=None, lse=None):
+    """Merge R partial decodes by their log-sum-exp (fa_decode_merge).
+    o_parts float32 [R,B,Hq,d] and lse_parts float32 [R,B,Hq]; each may have
+    any stride along R (e.g. views into one packed all-gather buffer) but must
+    be contiguous within a partial.  Returns O bf16 [B,Hq,d], LSE [B,Hq]."""
+    lib = load_library()
+    R, B, Hq, d = o_parts.shape
+    dev = o_parts.device
+    for n, t in (("o_parts", o_parts), ("lse_parts", lse_parts)):
+        if t.device.type != "cuda" or t.device != dev:
+            raise ValueError(f"{n} must be on {dev}")
+        if t.dtype != torch.float32:
+            raise TypeError(f"{n} must be float32")
+        if not t[0].is_contiguous():
+            raise ValueError(f"{n} must be contiguous within a partial")
+    if tuple(lse_parts.shape) != (R, B, Hq):
+        raise ValueError(f"lse_parts has shape {tuple(lse_parts.shape)}, expected {(R, B, Hq)}")
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_dev("out", out, torch.bfloat16, dev)
+    _check_dev("lse", lse, torch.float32, dev)
+    st = lib.fa_decode_merge(_ptr(o_parts), o_parts.stride(0), _ptr(lse_parts), lse_parts.stride(0), _ptr(out),
+                             _ptr(lse), R, B, Hq, d, _stream_ptr(dev))
+    _raise("fa_decode_merge", st)
     return out, lse
 
 

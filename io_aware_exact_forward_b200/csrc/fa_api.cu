@@ -450,9 +450,10 @@ size_t fa_decode_workspace_bytes(int B, int Hq, int Tk_max, int d, int chunk) {
 
 }  // extern "C"
 
+// `o` receives bf16 O, or, when `o32` is non-null instead, fp32 O.
 static int decode_impl(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k, void* o,
-                       float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tk_max, int d,
-                       float scale, int chunk, int window, void* stream) {
+                       float* o32, float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tk_max,
+                       int d, float scale, int chunk, int window, void* stream) {
   if (B < 0 || Hq < 1 || Hkv < 1 || Tk_max < 0 || Hq % Hkv != 0 || !isfinite(scale))
     return FA_ERR_INVALID_ARG;
   if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
@@ -462,9 +463,9 @@ static int decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   if (chunk < 64 || chunk % 64 != 0 || chunk * G > 4096) return FA_ERR_INVALID_ARG;
   if ((int64_t)Tk_max > (1 << 30) || (int64_t)B * Hq > (1 << 30)) return FA_ERR_INVALID_ARG;
   if (B == 0) return FA_OK;
-  if (!q || !seqlens_k || !o || !lse || (Tk_max > 0 && (!k_cache || !v_cache)))
+  if (!q || !seqlens_k || (!o == !o32) || !lse || (Tk_max > 0 && (!k_cache || !v_cache)))
     return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) ||
+  if (!aligned16(q) || !aligned16(o ? o : o32) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) ||
       (Tk_max > 0 && (!aligned16(k_cache) || !aligned16(v_cache))))
     return FA_ERR_ALIGNMENT;
   const size_t need = fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk);
@@ -485,6 +486,7 @@ static int decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   p.ws_o = reinterpret_cast<float*>(ws);
   p.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + round256((size_t)B * Hq * n * d * 4));
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.o32 = o32;
   p.lse = lse;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tk_max = Tk_max; p.chunk = chunk; p.nchunk = (int)n;
   p.n_items = (int)((size_t)B * Hkv * n);
@@ -529,16 +531,54 @@ extern "C" {
 int fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
                       void* o, float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv,
                       int Tk_max, int d, float scale, int chunk, void* stream) {
-  return decode_impl(q, k_cache, v_cache, seqlens_k, o, lse, ws, ws_bytes, B, Hq, Hkv, Tk_max, d, scale, chunk, 0,
-                     stream);
+  return decode_impl(q, k_cache, v_cache, seqlens_k, o, nullptr, lse, ws, ws_bytes, B, Hq, Hkv, Tk_max, d, scale,
+                     chunk, 0, stream);
+}
+
+int fa_decode_splitkv_partial(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
+                              float* o, float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv,
+                              int Tk_max, int d, float scale, int chunk, void* stream) {
+  return decode_impl(q, k_cache, v_cache, seqlens_k, nullptr, o, lse, ws, ws_bytes, B, Hq, Hkv, Tk_max, d, scale,
+                     chunk, 0, stream);
+}
+
+int fa_decode_merge(const float* o_parts, size_t o_stride, const float* lse_parts, size_t lse_stride, void* o,
+                    float* lse, int R, int B, int Hq, int d, void* stream) {
+  if (R < 1 || R > (1 << 20) || B < 0 || Hq < 1 || (int64_t)B * Hq > (1 << 30)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)B * Hq;
+  if (rows == 0) return FA_OK;
+  if (!o_parts || !lse_parts || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (R > 1 && (o_stride < rows * d || lse_stride < rows)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(o) || (o_stride & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse_parts) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGNMENT;
+  int st = device_setup();
+  if (st) return st;
+  MergeParams p;
+  p.o_parts = o_parts;
+  p.lse_parts = lse_parts;
+  p.o_stride = o_stride;
+  p.lse_stride = lse_stride;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.R = R;
+  p.rows = (int)rows;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+  if (d == 64)
+    fa_decode_merge_kernel<64><<<blocks, 256, 0, s>>>(p);
+  else
+    fa_decode_merge_kernel<128><<<blocks, 256, 0, s>>>(p);
+  return launch_status();
 }
 
 int fa_decode_splitkv_window(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
                              void* o, float* lse, void* ws, size_t ws_bytes, int B, int Hq, int Hkv,
                              int Tk_max, int d, float scale, int chunk, int window, void* stream) {
   if (window < 1) return FA_ERR_INVALID_ARG;
-  return decode_impl(q, k_cache, v_cache, seqlens_k, o, lse, ws, ws_bytes, B, Hq, Hkv, Tk_max, d, scale, chunk,
-                     window, stream);
+  return decode_impl(q, k_cache, v_cache, seqlens_k, o, nullptr, lse, ws, ws_bytes, B, Hq, Hkv, Tk_max, d, scale,
+                     chunk, window, stream);
 }
 
 int fa_check(void* stream) {

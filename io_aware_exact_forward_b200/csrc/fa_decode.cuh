@@ -40,6 +40,7 @@ struct DecodeParams {
   float* ws_o;               // [B][Hq][nchunk][d]
   float* ws_lse;             // [B][Hq][nchunk]
   __nv_bfloat16* o;          // [B][Hq][d]
+  float* o32;                // non-null: O goes here in fp32 [B][Hq][d] instead of to `o`
   float* lse;                // [B][Hq]
   int B, Hq, Hkv, Tk_max, chunk, nchunk;
   int n_items;               // B * Hkv * nchunk (items past a sequence's end are skipped)
@@ -345,6 +346,22 @@ fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
   }
 }
 
+// One output row of D values, D/32 consecutive ones per lane: bf16 into `o`,
+// or fp32 into `o32` when the caller asked for partials to merge later.
+template <int D>
+__device__ __forceinline__ void store_row(const DecodeParams& p, int row, int lane, const float (&acc)[D / 32]) {
+  constexpr int E = D / 32;
+  if (p.o32) {
+    float* dst = p.o32 + (size_t)row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) *reinterpret_cast<float2*>(dst + e) = make_float2(acc[e], acc[e + 1]);
+  } else {
+    __nv_bfloat16* dst = p.o + (size_t)row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
+  }
+}
+
 // Separate merge of the chunk partials: one warp per (sequence, query head).
 template <int D>
 __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const __grid_constant__ DecodeParams p) {
@@ -394,9 +411,7 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const __grid_con
     for (int e = 0; e < E; ++e) acc[e] = fmaf(w, o_c[(size_t)cc * D + lane * E + e], acc[e]);
   }
   if (lane == 0) p.lse[gw] = lse;
-  __nv_bfloat16* dst = p.o + (size_t)gw * D + lane * E;
-#pragma unroll
-  for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
+  store_row<D>(p, gw, lane, acc);
 }
 
 // Sequences with no cached key (seqlen 0) get O = 0 and LSE = -inf; every
@@ -408,11 +423,71 @@ __global__ void __launch_bounds__(256) fa_decode_empty_kernel(const __grid_const
   if (gw >= p.B * p.Hq) return;
   const int b = gw / p.Hq;
   if (p.seqlens[b] > 0) return;
-  constexpr int E = D / 32;
-  __nv_bfloat16* dst = p.o + (size_t)gw * D + lane * E;
+  float zero[D / 32];
 #pragma unroll
-  for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = 0u;
+  for (int e = 0; e < D / 32; ++e) zero[e] = 0.f;
+  store_row<D>(p, gw, lane, zero);
   if (lane == 0) p.lse[gw] = -INFINITY;
+}
+
+// Merge of per-device partials (context-parallel decode): device r decoded
+// its own share of every sequence's keys into a normalised fp32 O_r and
+// LSE_r; the full result is
+//   LSE = log sum_r e^{LSE_r},  O = sum_r e^{LSE_r - LSE} O_r,
+// the chunk merge above with devices in place of chunks.  A device whose
+// share of a sequence is empty contributes LSE_r = -inf and is skipped; a
+// row no device saw a key of gets O = 0 and LSE = -inf.
+struct MergeParams {
+  const float* o_parts;    // [R] blocks of [rows][d], `o_stride` floats apart
+  const float* lse_parts;  // [R] blocks of [rows], `lse_stride` floats apart
+  size_t o_stride, lse_stride;
+  __nv_bfloat16* o;        // [rows][d]
+  float* lse;              // [rows]
+  int R, rows;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) fa_decode_merge_kernel(const __grid_constant__ MergeParams p) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= p.rows) return;
+  constexpr int E = D / 32;
+  constexpr float kLog2e = 1.4426950408889634f;
+  float mx = -INFINITY;
+  for (int r = lane; r < p.R; r += 32) mx = fmaxf(mx, p.lse_parts[(size_t)r * p.lse_stride + row]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  if (mx == -INFINITY) {
+    __nv_bfloat16* dst = p.o + (size_t)row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = 0u;
+    if (lane == 0) p.lse[row] = -INFINITY;
+    return;
+  }
+  float sum = 0.f;
+  for (int r = lane; r < p.R; r += 32) sum += ex2_approx((p.lse_parts[(size_t)r * p.lse_stride + row] - mx) * kLog2e);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  const float lse = mx + logf(sum);
+  for (int r = 0; r < p.R; ++r) {
+    const float l = p.lse_parts[(size_t)r * p.lse_stride + row];
+    if (l == -INFINITY) continue;  // same value in every lane: no divergence
+    const float w = ex2_approx((l - lse) * kLog2e);
+    const float* src = p.o_parts + (size_t)r * p.o_stride + (size_t)row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
+      const float2 x = *reinterpret_cast<const float2*>(src + e);
+      acc[e] = fmaf(w, x.x, acc[e]);
+      acc[e + 1] = fmaf(w, x.y, acc[e + 1]);
+    }
+  }
+  if (lane == 0) p.lse[row] = lse;
+  __nv_bfloat16* dst = p.o + (size_t)row * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
 }
 
 }  // namespace fa

@@ -119,3 +119,25 @@ def test_decode_window_rejects_bad_window_on_host():
         assert lib.fa_decode_splitkv_window(*([NULL] * 6), NULL, 0, 2, 32, 8, 1024, 128, 0.1, 256, w, NULL) == 1
     # otherwise the same checks as fa_decode_splitkv (G = 16 unsupported)
     assert lib.fa_decode_splitkv_window(*([NULL] * 6), NULL, 0, 2, 32, 2, 1024, 128, 0.1, 256, 8, NULL) == 2
+
+
+def test_context_parallel_decode_argument_checks():
+    lib = fa.load_library()
+    # partial decode: the same checks as fa_decode_splitkv; a null fp32 output is rejected
+    assert lib.fa_decode_splitkv_partial(*([NULL] * 6), NULL, 0, 2, 32, 2, 1024, 128, 0.1, 256, NULL) == 2
+    assert lib.fa_decode_splitkv_partial(*([NULL] * 6), NULL, 0, 2, 32, 8, 1024, 128, 0.1, 256, NULL) == 1
+    # merge: (o_parts, o_stride, lse_parts, lse_stride, o, lse, R, B, Hq, d, stream)
+    assert lib.fa_decode_merge(NULL, 0, NULL, 0, NULL, NULL, 0, 2, 4, 64, NULL) == 1     # R = 0
+    assert lib.fa_decode_merge(NULL, 0, NULL, 0, NULL, NULL, 2, 2, 4, 96, NULL) == 2     # head dim
+    assert lib.fa_decode_merge(NULL, 0, NULL, 0, NULL, NULL, 2, 0, 4, 64, NULL) == 0     # no rows: no-op
+    assert lib.fa_decode_merge(NULL, 0, NULL, 0, NULL, NULL, 2, 2, 4, 64, NULL) == 1     # null pointers
+    buf = (ctypes.c_uint8 * 256)()
+    base = ctypes.addressof(buf) + (16 - ctypes.addressof(buf) % 16) % 16
+    al = ctypes.c_void_p(base)
+    rows, d = 2 * 4, 64
+    # strides shorter than one partial
+    assert lib.fa_decode_merge(al, rows * d - 4, al, rows, al, al, 2, 2, 4, d, NULL) == 1
+    assert lib.fa_decode_merge(al, rows * d, al, rows - 1, al, al, 2, 2, 4, d, NULL) == 1
+    # O stride not a multiple of 4 floats, or a misaligned O block
+    assert lib.fa_decode_merge(al, rows * d + 2, al, rows, al, al, 2, 2, 4, d, NULL) == 3
+    assert lib.fa_decode_merge(ctypes.c_void_p(base + 8), rows * d, al, rows, al, al, 2, 2, 4, d, NULL) == 3

@@ -42,6 +42,12 @@ Readings where the pages are silent (each is also listed in the design notes):
   query i sees key j iff i + (Tk - Tq) - W < j <= i + (Tk - Tq), i.e. its own
   diagonal key and the W - 1 keys before it.  W >= Tk is the causal mask.
 
+The FP8 forward (FlashAttention-3's low-precision path, named in [FA §"In
+practice"]) is checked against ``attention_forward_e4m3``: exact attention on
+the dequantised E4M3 inputs.  E4M3 is decoded here from the format's
+published definition (the OCP 8-bit floating-point specification, "FP8
+Formats for Deep Learning", Micikevicius et al. 2022), not by a library.
+
 Layouts follow the library: q, o, dq are [B, Tq, Hq, d]; k, v, dk, dv are
 [B, Tk, Hkv, d]; lse is [B, Hq, Tq].  All arrays are float64.
 """
@@ -63,6 +69,9 @@ __all__ = [
     "online_softmax_row",
     "combine_partials",
     "merge_partials",
+    "e4m3_value",
+    "e4m3_decode",
+    "attention_forward_e4m3",
     "brute_force_row",
 ]
 
@@ -219,6 +228,43 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, window=None):
             dk[b, :, g] += bk
             dv[b, :, g] += bv
     return dq, dk, dv
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one E4M3 byte: bit 7 the sign, bits 3-6 the exponent field E
+    (bias 7), bits 0-2 the mantissa field M.  E > 0: (1 + M/8) * 2^(E - 7);
+    E = 0: subnormal (M/8) * 2^-6; E = 15 with M = 7 is NaN (the format has
+    no infinities, so E = 15 with M < 7 are ordinary values up to 448)."""
+    code = int(code) & 0xFF
+    sign = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 15 and m == 7:
+        return math.nan
+    if e == 0:
+        return sign * (m / 8.0) * 2.0 ** -6
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+_E4M3_TABLE = None
+
+
+def e4m3_decode(codes):
+    """Element-wise ``e4m3_value`` of an array of E4M3 bytes (uint8)."""
+    global _E4M3_TABLE
+    if _E4M3_TABLE is None:
+        _E4M3_TABLE = np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+def attention_forward_e4m3(q8, k8, v8, q_descale, k_descale, v_descale, scale: float, causal: bool):
+    """Exact attention on E4M3 inputs: each tensor's values are its decoded
+    codes times its descale factor; then ``attention_forward``.  q8, k8, v8
+    are uint8 code arrays in the library's layouts."""
+    q = e4m3_decode(q8) * float(q_descale)
+    k = e4m3_decode(k8) * float(k_descale)
+    v = e4m3_decode(v8) * float(v_descale)
+    return attention_forward(q, k, v, scale, causal)
 
 
 def decode_forward(q, k_cache, v_cache, seqlens, scale: float, pairs=None, window=None):

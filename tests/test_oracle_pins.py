@@ -512,3 +512,49 @@ def test_window_decode_is_last_prefill_row():
             Ob, Lb = oracle.head_forward(q[b, h][None, :], kc[b, lo:n, g], vc[b, lo:n, g], 0.3, False)
             np.testing.assert_allclose(O[b, h], Ob[0], rtol=1e-13, atol=1e-15)
             assert math.isclose(LSE[b, h], Lb[0], rel_tol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# E4M3 decoding and the FP8 forward's reference
+# ---------------------------------------------------------------------------
+
+def test_e4m3_closed_forms():
+    v = oracle.e4m3_value
+    assert v(0x38) == 1.0 and v(0xB8) == -1.0          # E = 7, M = 0
+    assert v(0x7E) == 448.0 and v(0xFE) == -448.0      # the largest finite value
+    assert v(0x08) == 2.0 ** -6                        # the smallest normal
+    assert v(0x01) == 2.0 ** -9 and v(0x07) == 7 * 2.0 ** -9   # subnormals
+    assert v(0x00) == 0.0 and math.copysign(1.0, v(0x80)) == -1.0
+    assert math.isnan(v(0x7F)) and math.isnan(v(0xFF))
+    assert v(0x78) == 256.0 and v(0x3C) == 1.5 and v(0x40) == 2.0
+    vals = [v(c) for c in range(0x7F)]
+    assert all(a < b for a, b in zip(vals, vals[1:]))  # codes 0..126 increase
+
+
+def test_e4m3_decode_matches_torch_conversion():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = oracle.e4m3_decode(codes.numpy())
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(ours)) and nan.sum() == 2
+    np.testing.assert_array_equal(ours[~nan], ref[~nan])
+
+
+def test_e4m3_attention_descale_factors():
+    """The factors act where the definition puts them: q and k scale the
+    scores (doubling q's equals doubling the softmax scale), v scales O
+    linearly and leaves LSE alone."""
+    rng = np.random.default_rng(8)
+    B, T, H, d = 1, 9, 2, 4
+    q8, k8, v8 = (rng.integers(0, 0x7F, size=(B, T, H, d)) | (rng.integers(0, 2, size=(B, T, H, d)) << 7)
+                  for _ in range(3))
+    O, L = oracle.attention_forward_e4m3(q8, k8, v8, 0.01, 0.02, 0.5, 0.3, True)
+    O2, L2 = oracle.attention_forward_e4m3(q8, k8, v8, 0.02, 0.02, 1.5, 0.3, True)
+    O3, L3 = oracle.attention_forward_e4m3(q8, k8, v8, 0.01, 0.02, 1.5, 0.6, True)
+    np.testing.assert_allclose(O2, O3, rtol=1e-13)
+    np.testing.assert_allclose(L2, L3, rtol=1e-13)
+    Ob, Lb = oracle.attention_forward_e4m3(q8, k8, v8, 0.01, 0.02, 1.5, 0.3, True)
+    np.testing.assert_allclose(Ob, 3.0 * O, rtol=1e-13)
+    np.testing.assert_array_equal(Lb, L)
+    # first causal row sees key 0 only: O = that value row
+    np.testing.assert_allclose(O[0, 0], oracle.e4m3_decode(v8[0, 0]) * 0.5, rtol=1e-15)

@@ -15,6 +15,11 @@ Recipe (the same for every consumer):
 * Outlier keys (the long-context GQA workload): after dO, one ``randperm`` of
   the T token positions per (b, kv head); the first round(0.01 * T) positions
   have all d entries of K multiplied by 4 (exact in bf16).
+* E4M3 prefill (the FP8 forward): the same Q, K, V draws as prefill (outlier
+  keys included), each tensor then quantised with one factor
+  descale = amax(|x|) / 448 as code = E4M3(x / descale), rounded to nearest
+  by torch's float8_e4m3fn conversion.  The codes and the three factors are
+  the inputs; both sides read the same codes.
 * Decode: seqlens ~ integer-uniform on [1024, 32768] inclusive, then q
   [B, Hq, d], then per sequence b the K and V cache rows [Tk_max, Hkv, d], all
   fp32 N(0,1) rounded to bf16.  Only the first seqlens[b] rows are read.
@@ -33,7 +38,7 @@ from dataclasses import dataclass, field, replace
 import numpy as np
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "prefill_inputs", "decode_inputs", "to_f64"]
+__all__ = ["Workload", "WORKLOADS", "prefill_inputs", "prefill_inputs_e4m3", "decode_inputs", "to_f64"]
 
 
 @dataclass(frozen=True)
@@ -109,6 +114,32 @@ def prefill_inputs(w: Workload, device="cpu", seed=None, Tq=None, Tk=None):
     out = {n: t.to(torch.bfloat16).contiguous() for n, t in
            (("q", q), ("k", k), ("v", v), ("do", do))}
     out["outlier_rows"] = outliers
+    return out
+
+
+def prefill_inputs_e4m3(w: Workload, device="cpu", seed=None, Tq=None, Tk=None):
+    """E4M3 codes of Q, K, V (torch.float8_e4m3fn, BTHD) and their descale
+    factors, from the fp32 draws of ``prefill_inputs`` (same seed, same
+    outlier keys) quantised per tensor with amax / 448."""
+    Tq = w.T if Tq is None else Tq
+    Tk = w.T if Tk is None else Tk
+    g = _gen(device, w.seed if seed is None else seed)
+    q = torch.randn((w.B, Tq, w.Hq, w.d), generator=g, device=device)
+    k = torch.randn((w.B, Tk, w.Hkv, w.d), generator=g, device=device)
+    v = torch.randn((w.B, Tk, w.Hkv, w.d), generator=g, device=device)
+    if w.outlier_frac > 0 and Tk > 0:
+        torch.randn((w.B, Tq, w.Hq, w.d), generator=g, device=device)   # dO's draw, to keep the stream aligned
+        n_out = int(round(w.outlier_frac * Tk))
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                idx = torch.randperm(Tk, generator=g, device=device)[:n_out]
+                k[b, idx, h, :] *= w.outlier_scale
+    out = {}
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        amax = float(t.abs().max()) if t.numel() else 1.0
+        descale = amax / 448.0 if amax > 0 else 1.0
+        out[n] = (t / descale).to(torch.float8_e4m3fn).contiguous()
+        out[n + "_descale"] = descale
     return out
 
 

@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--window", type=int, default=None,
                     help="sliding window of that many keys (prefill: implies causal; decode: last keys)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="prefill, d = 128 only: the E4M3 forward (fa_forward_fp8) alone")
     ap.add_argument("--cp", action="store_true",
                     help="decode only: context-parallel, every sequence's cache cut into one share per GPU")
     ap.add_argument("--batch", type=int, default=None,
@@ -680,6 +682,133 @@ def run_decode(args, w, rank, world, dist):
     return 0
 
 
+def run_fp8_forward(args, w, rank, world, dist):
+    """The E4M3 forward on a d = 128 prefill workload: one step is one
+    fa_forward_fp8 launch over the whole batch (Q, K, V codes resident).
+    value is algorithmic TFLOP/s (4 B Hq d pairs); the roofline denominator is
+    the measured bf16 peak times 2, the nominal E4M3:bf16 ratio of the tensor
+    cores (4.5 : 2.25 PFLOP/s dense)."""
+    import ctypes
+    import torch
+    import io_aware_exact_forward_b200 as fa
+    from workloads import prefill_inputs_e4m3
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = fa.load_library()
+    inp = prefill_inputs_e4m3(w, device=dev, seed=w.seed + rank)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    qs, ks, vs = inp["q_descale"], inp["k_descale"], inp["v_descale"]
+    B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
+    o = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    P = ctypes.c_void_p
+    stream = torch.cuda.current_stream(dev)
+    sp = P(stream.cuda_stream)
+    args_c = (P(q.data_ptr()), P(k.data_ptr()), P(v.data_ptr()), qs, ks, vs, P(o.data_ptr()), P(lse.data_ptr()),
+              B, Hq, Hkv, T, T, d, w.scale, int(w.causal), sp)
+
+    def step():
+        st = lib.fa_forward_fp8(*args_c)
+        if st != 0:
+            raise RuntimeError(f"fa_forward_fp8: {fa.STATUS.get(st, st)}")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    # L2 is flushed between timed launches by writing a 256 MiB buffer
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        for s_ in range(args.steps):
+            flush.fill_(s_ & 0xFF)
+            evs[s_][0].record(stream)
+            step()
+            evs[s_][1].record(stream)
+        barrier()
+    if lib.fa_check(sp) != 0:
+        raise RuntimeError("device status set during the timed region")
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), dist, dev)
+    f_fwd, _ = flops(w)
+    value = job_rate(f_fwd, world, args.steps, ms) / 1e12
+    peaks = load_peaks()
+    peak = 2.0 * peaks["bf16_tflops"]
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            fa.forward_fp8(q, k, v, qs, ks, vs, scale=w.scale, causal=w.causal, out=o, lse=lse)
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        f1.record(stream)
+        barrier()
+        e_ms = max_over_ranks(f0.elapsed_time(f1), dist, dev)
+        e2e = {"value": job_rate(f_fwd, world, args.e2e_steps, e_ms) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hlse.numel() * hlse.element_size(),
+               "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        G = Hq // Hkv
+        per_head = f_fwd / (B * Hq)
+        qc, kc, vc = (t.view(torch.uint8).cpu() for t in (q, k, v))
+        done, t0 = 0, time.perf_counter()
+        for h in range(Hq):
+            oracle.attention_forward_e4m3(qc[:1, :, h:h + 1].numpy(), kc[:1, :, h // G:h // G + 1].numpy(),
+                                          vc[:1, :, h // G:h // G + 1].numpy(), qs, ks, vs, w.scale, w.causal)
+            done += 1
+            if time.perf_counter() - t0 >= args.cpu_seconds:
+                break
+        dt = time.perf_counter() - t0
+        cpu = {"value": done * per_head / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"float64 oracle forward on E4M3 inputs, {done} of {B * Hq} heads of {w.name} "
+                         f"({dt:.1f} s; same algorithmic FLOP count as the GPU metric)"}
+    if rank == 0:
+        line = {
+            "metric": "attention forward TFLOPS (E4M3 inputs, 1xB200) and % of dense E4M3 tensor peak",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
+                       "inputs": "E4M3 codes, per-tensor amax/448 factors", "l2": "256 MiB flush between launches",
+                       "seed": w.seed},
+            "roofline": {"kernel": "fa_fwd_kernel<128, true>", "bound": "tensor", "achieved": value / world,
+                         "peak": peak, "unit": "TFLOP/s", "frac": value / world / peak,
+                         "peak_source": f"{peaks['source']} bf16 dense (burst) x 2, the nominal E4M3:bf16 ratio",
+                         "traffic": None, "algorithmic_per_launch": f_fwd},
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_decode_cp(args, w, rank, world, dist):
     """Context-parallel decode of the same batch: every sequence's cache is
     cut into `world` contiguous shares and rank r holds share r.  One step is
@@ -822,6 +951,9 @@ def main():
     dist = None
     if args.impl == "reference":
         return run_reference(args, w, rank)
+    if args.fp8 and (w.decode or w.d != 128 or w.window):
+        print("--fp8 applies to the d = 128 prefill workloads without a window", file=sys.stderr)
+        return 2
     if args.cp and (not w.decode or w.window):
         print("--cp applies to the decode workload without a window", file=sys.stderr)
         return 2
@@ -836,6 +968,8 @@ def main():
         tdist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
         dist = tdist
     try:
+        if args.fp8:
+            return run_fp8_forward(args, w, rank, world, dist)
         if w.decode and args.cp:
             return run_decode_cp(args, w, rank, world, dist)
         if w.decode:

@@ -99,6 +99,25 @@ int fa_forward_window(const void* q, const void* k, const void* v, void* o, floa
                       void* stream);
 
 /*
+ * fa_forward_fp8 -- fa_forward with 8-bit inputs: the low-precision forward
+ * that "FlashAttention" (interview track, "In practice") lists for FA3, here
+ * on B200's kind::f8f6f4 tensor-core MMAs.
+ *   q, k, v   E4M3 (OCP FP8: 1 sign, 4 exponent bits with bias 7, 3 mantissa
+ *             bits), one byte per element, layouts as fa_forward.
+ *   q_descale, k_descale, v_descale  the factor that turns each tensor's
+ *             codes into its values (value = code * descale), finite and > 0.
+ *   o, lse    as fa_forward (bf16 O, fp32 LSE of the scaled scores).
+ * The result is attention on the dequantised inputs, with P rounded to E4M3
+ * before P V (the row sums l use the unrounded P); that rounding makes O
+ * differ from exact attention by up to a few percent on rows with few keys
+ * (3 mantissa bits), much less on long rows.  d must be 128
+ * (FA_ERR_UNSUPPORTED otherwise); other arguments and errors as fa_forward.
+ */
+int fa_forward_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                   float v_descale, void* o, float* lse, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+                   float scale, int causal, void* stream);
+
+/*
  * Bytes of device workspace fa_backward needs: an fp32 dQ accumulator
  * [B,Tq,Hq,d], the fp32 row terms D_i = sum_c dO_ic O_ic and the LSE in log2
  * units, each [B,Hq,Tq_pad] with Tq_pad = Tq rounded up to 128; every piece

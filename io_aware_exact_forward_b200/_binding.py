@@ -33,6 +33,7 @@ SIGNATURES = {
     "fa_version": (_c_int, []),
     "fa_forward": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_forward_window": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_forward_fp8": (_c_int, [_vp] * 3 + [_c_float] * 3 + [_vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_workspace_bytes": (_c_size, [_c_int] * 6),
     "fa_backward": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_window": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
@@ -131,6 +132,31 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, window=None):
         st = lib.fa_forward_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tk, d,
                                    float(scale), int(window), _stream_ptr(dev))
         _raise("fa_forward_window", st)
+    return out, lse
+
+
+def forward_fp8(q, k, v, q_descale, k_descale, v_descale, scale=None, causal=False, out=None, lse=None):
+    """O, LSE of attention on E4M3 inputs (fa_forward_fp8).  q [B,Tq,Hq,128],
+    k/v [B,Tk,Hkv,128] torch.float8_e4m3fn (CUDA); the descale factors map
+    codes to values.  O is bf16, LSE fp32 [B,Hq,Tq]."""
+    lib = load_library()
+    B, Tq, Hq, d = q.shape
+    Tk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_dev(n, t, torch.float8_e4m3fn, dev)
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty((B, Tq, Hq, d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=dev)
+    _check_dev("out", out, torch.bfloat16, dev)
+    _check_dev("lse", lse, torch.float32, dev)
+    st = lib.fa_forward_fp8(_ptr(q), _ptr(k), _ptr(v), float(q_descale), float(k_descale), float(v_descale),
+                            _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tk, d, float(scale), int(bool(causal)),
+                            _stream_ptr(dev))
+    _raise("fa_forward_fp8", st)
     return out, lse
 
 

@@ -49,15 +49,17 @@ static EncodeTiledFn encode_fn() {
 // 4-D bf16 tensor [n3][n2][n1][n0] (n0 contiguous) with box {64, 1, box_rows, 1}
 // along (n0, n1, n2, n3) and the 128-byte swizzle, or no swizzle when
 // `swizzle` is false (then box_inner elements along n0).
+// elt = 2: bf16 elements; elt = 1: 8-bit (E4M3) elements.
 static int make_tmap_4d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
-                        uint64_t n3, uint32_t box_inner, uint32_t box_rows, bool swizzle) {
+                        uint64_t n3, uint32_t box_inner, uint32_t box_rows, bool swizzle, int elt = 2) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return FA_ERR_CUDA;
   const cuuint64_t dims[4] = {n0, n1, n2, n3};
-  const cuuint64_t strides[3] = {n0 * 2, n0 * n1 * 2, n0 * n1 * n2 * 2};
+  const cuuint64_t strides[3] = {n0 * elt, n0 * n1 * elt, n0 * n1 * n2 * elt};
   const cuuint32_t box[4] = {box_inner, 1, box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+  CUresult r = fn(m, elt == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -123,6 +125,7 @@ static int device_setup_impl() {
   int st = FA_OK;
   if (!st) st = set_smem(fa_fwd_kernel<64>, FwdCfg<64>::SMEM_BYTES);
   if (!st) st = set_smem(fa_fwd_kernel<128>, FwdCfg<128>::SMEM_BYTES);
+  if (!st) st = set_smem(fa_fwd_kernel<128, true>, FwdCfg<128, true>::SMEM_BYTES);
   if (!st) st = bwd_setup();
   if (!st) st = decode_setup();
   return st;
@@ -201,11 +204,15 @@ int fa_version(void) { return 100; }
 }  // extern "C"
 
 // window > 0: sliding window of that many keys (the caller passes causal = 1).
+// f8: q, k, v are E4M3; `qk_factor` multiplies the scores' scale and
+// `o_scale` the output (the dequantising factors).
 static int forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                        int Hkv, int Tq, int Tk, int d, float scale, int causal, int window, void* stream) {
+                        int Hkv, int Tq, int Tk, int d, float scale, int causal, int window, void* stream,
+                        bool f8 = false, float qk_factor = 1.f, float o_scale = 1.f) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
   if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
+  if (f8 && d != 128) return FA_ERR_UNSUPPORTED;
   if (B == 0 || Tq == 0) return FA_OK;
   if (!q || !o || !lse || (Tk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || (Tk > 0 && (!aligned16(k) || !aligned16(v))))
@@ -214,16 +221,18 @@ static int forward_impl(const void* q, const void* k, const void* v, void* o, fl
   if (st) return st;
   FwdParams p;
   memset(&p, 0, sizeof(p));
-  st = make_tmap_4d(&p.tm_q, q, d, Hq, Tq, B, 64, 128, true);
-  if (!st && Tk > 0) st = make_tmap_4d(&p.tm_k, k, d, Hkv, Tk, B, 64, 128, true);
-  if (!st && Tk > 0) st = make_tmap_4d(&p.tm_v, v, d, Hkv, Tk, B, 64, 128, true);
+  const int elt = f8 ? 1 : 2, box_inner = 128 / elt;  // one 128-byte swizzle row per box
+  st = make_tmap_4d(&p.tm_q, q, d, Hq, Tq, B, box_inner, 128, true, elt);
+  if (!st && Tk > 0) st = make_tmap_4d(&p.tm_k, k, d, Hkv, Tk, B, box_inner, 128, true, elt);
+  if (!st && Tk > 0) st = make_tmap_4d(&p.tm_v, v, d, Hkv, Tk, B, box_inner, 128, true, elt);
   if (st) return st;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tq = Tq; p.Tk = Tk;
   p.causal = causal;
   p.window = window;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * qk_factor * 1.4426950408889634f;
+  p.o_scale = o_scale;
   p.n_mblocks = (Tq + 255) / 256;
   p.n_items = B * Hq * p.n_mblocks;
   p.wait_limit_ns = kWaitLimitNs;
@@ -234,7 +243,9 @@ static int forward_impl(const void* q, const void* k, const void* v, void* o, fl
   if ((st = sm_count(&nsm))) return st;
   dim3 grid(causal ? p.n_items : std::min(p.n_items, nsm));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
+  if (f8)
+    fa_fwd_kernel<128, true><<<grid, FwdCfg<128, true>::THREADS, FwdCfg<128, true>::SMEM_BYTES, s>>>(p);
+  else if (d == 64)
     fa_fwd_kernel<64><<<grid, FwdCfg<64>::THREADS, FwdCfg<64>::SMEM_BYTES, s>>>(p);
   else
     fa_fwd_kernel<128><<<grid, FwdCfg<128>::THREADS, FwdCfg<128>::SMEM_BYTES, s>>>(p);
@@ -252,6 +263,16 @@ int fa_forward_window(const void* q, const void* k, const void* v, void* o, floa
                       int Hkv, int Tq, int Tk, int d, float scale, int window, void* stream) {
   if (window < 1) return FA_ERR_INVALID_ARG;
   return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, d, scale, 1, window, stream);
+}
+
+int fa_forward_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                   float v_descale, void* o, float* lse, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+                   float scale, int causal, void* stream) {
+  for (float f : {q_descale, k_descale, v_descale})
+    if (!(f > 0.f) || !isfinite(f)) return FA_ERR_INVALID_ARG;
+  if (!isfinite(scale * q_descale * k_descale)) return FA_ERR_INVALID_ARG;
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0, stream, true,
+                      q_descale * k_descale, v_descale);
 }
 
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }

@@ -31,6 +31,15 @@
 // The two softmax warpgroups alternate with the tensor core: while one
 // computes exponentials the other's MMAs run.
 //
+// FP8 variant (F8 = true, d = 128): Q, K and V are E4M3 with one dequantising
+// factor per tensor, the two products run as kind::f8f6f4 MMAs (twice the bf16
+// rate), and P is rounded to E4M3 for P V (32 tensor-memory columns over S),
+// as FlashAttention-3's low-precision forward does ("FlashAttention",
+// interview track, "In practice").  The q and k factors fold into the
+// exponent's scale, the v factor into the epilogue's 1 / l; l itself sums the
+// unrounded fp32 p.  P goes to shared memory (16 KB per query tile), so that
+// the next S overlaps the softmax as in the d = 64 kernel.
+//
 // The rescale is lazy: a row keeps its reference maximum until the running
 // maximum exceeds it by more than 8 (log2 units), so exponentials stay below
 // 2^8.  l and u always share one reference, so the result is the same
@@ -42,7 +51,7 @@
 namespace fa {
 
 struct FwdParams {
-  CUtensorMap tm_q;   // [B][Tq][Hq][d] bf16, box {64, 1, 128, 1}, 128-byte swizzle
+  CUtensorMap tm_q;   // [B][Tq][Hq][d] bf16 (E4M3), box {64 (128), 1, 128, 1}, 128-byte swizzle
   CUtensorMap tm_k;   // [B][Tk][Hkv][d]
   CUtensorMap tm_v;
   __nv_bfloat16* o;   // [B][Tq][Hq][d]
@@ -50,23 +59,30 @@ struct FwdParams {
   int B, Hq, Hkv, Tq, Tk;
   int causal;
   int window;         // > 0: sliding window of that many keys (implies causal)
-  float scale_log2;   // scale * log2(e)
+  float scale_log2;   // scale * log2(e) (times the q and k factors for E4M3 inputs)
+  float o_scale;      // multiplies O = u / l: 1, or the v factor for E4M3 inputs
   int n_mblocks;      // ceil(Tq / 256): work items per (batch, head)
   int n_items;        // B * Hq * n_mblocks
   unsigned long long wait_limit_ns;
 };
 
-template <int D>
+template <int D, bool F8 = false>
 struct FwdCfg {
   static constexpr int BM = 128;                 // rows per query tile
   static constexpr int BN = 128;                 // keys per KV tile
-  static constexpr int NBOX = D / 64;            // 64-element swizzle boxes along d
+  static constexpr int ELT = F8 ? 1 : 2;         // bytes per element
+  static constexpr int BOX_ELEMS = 128 / ELT;    // elements per 128-byte swizzle row
+  static constexpr int NBOX = D / BOX_ELEMS;     // swizzle boxes along d
   static constexpr int BOX_BYTES = 128 * 128;    // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;
-  static constexpr int NSTAGE = (D == 64) ? 6 : 3;
+  static constexpr int KSTEP = 32 / ELT;         // K elements per MMA instruction (32 bytes)
+  static constexpr int NSTAGE = F8 ? 8 : (D == 64) ? 6 : 3;
   static constexpr int OFF_Q = 0;                // 2 buffers x (Q0, Q1)
   static constexpr int OFF_RING = 4 * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_RING + NSTAGE * TILE_BYTES;
+  // E4M3: P0, P1 (128 rows x 128 one-byte keys each) in shared memory
+  static constexpr int P_BYTES = BM * BN;
+  static constexpr int OFF_P = OFF_RING + NSTAGE * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_P + (F8 ? 2 * P_BYTES : 0);
   // q_full[2], q_empty[2], kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2],
   // p_full[2], o_final[2], mma_done, s_free[2], p_free[2]
   static constexpr int NBAR = 4 + 2 * NSTAGE + 2 + 2 + 2 + 1 + 4;
@@ -74,15 +90,17 @@ struct FwdCfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 320;
   static constexpr int TMEM_COLS = 512;
-  // d = 64: P gets its own tensor-memory columns (after S0, S1, O0, O1), so
-  // that the next S can be computed as soon as the softmax has loaded this
-  // one, overlapping the softmax; d = 128 has no room and writes P over S.
-  static constexpr bool SEP_P = (D == 64);
+  // P apart from S, so that the next S can be computed as soon as the softmax
+  // has loaded this one, overlapping the softmax: at d = 64 (bf16) in its own
+  // tensor-memory columns after S0, S1, O0, O1; with E4M3 (d = 128, tensor
+  // memory full) in shared memory, where one-byte P takes 16 KB per tile.
+  // bf16 at d = 128 has room in neither and writes P over S.
+  static constexpr bool SEP_P = (D == 64) || F8;
   // With SEP_P the ring holds (K_j, V_j) pairs with one barrier pair each.
   static constexpr int NPAIR = NSTAGE / 2;
   static constexpr int TM_P = 256 + 2 * D;       // P0, P1: 64 columns each (SEP_P)
-  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
-  static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
+  static constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(128, BN, 0, 0) : idesc_bf16_f32(128, BN, 0, 0);
+  static constexpr uint32_t IDESC_O = F8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
   static constexpr float RESCALE_THRESHOLD = 8.0f;
   // Pairs of S columns whose exponentials use exp2_poly2: 3 of every 8 at
   // d = 128, where the shared MUFU unit limits the softmax, 1 of every 8 at
@@ -91,6 +109,7 @@ struct FwdCfg {
     return D == 128 ? ((c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6) : ((c & 7) == 3);
   }
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+  static_assert(!F8 || D == 128, "the E4M3 forward is built for d = 128");
 };
 
 // One work item: two query tiles [m0, m0 + 256) of head h of batch b,
@@ -101,7 +120,7 @@ struct FwdItem {
 
 template <int D>
 __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D>;  // BM and BN are the same for both element types
   FwdItem it;
   // Query blocks of one (batch, head) are adjacent in item order, so they
   // share that head's K/V tiles through L2; within a head the heaviest
@@ -129,9 +148,9 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   return it;
 }
 
-template <int D>
+template <int D, bool F8 = false>
 __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -201,8 +220,10 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
         if (!ok) break;
         mbar_arrive_expect_tx(bar_q_full(qb), 2 * C::TILE_BYTES);
         for (int kb = 0; kb < C::NBOX; ++kb) {
-          tma_load_4d(q_addr(qb, 0) + kb * C::BOX_BYTES, &p.tm_q, bar_q_full(qb), kb * 64, it.h, it.m0, it.b);
-          tma_load_4d(q_addr(qb, 1) + kb * C::BOX_BYTES, &p.tm_q, bar_q_full(qb), kb * 64, it.h, it.m0 + C::BM, it.b);
+          tma_load_4d(q_addr(qb, 0) + kb * C::BOX_BYTES, &p.tm_q, bar_q_full(qb), kb * C::BOX_ELEMS, it.h, it.m0,
+                      it.b);
+          tma_load_4d(q_addr(qb, 1) + kb * C::BOX_BYTES, &p.tm_q, bar_q_full(qb), kb * C::BOX_ELEMS, it.h,
+                      it.m0 + C::BM, it.b);
         }
         for (int j = 0; j < it.n_kv && ok; ++j) {
           if constexpr (C::SEP_P) {
@@ -227,7 +248,7 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
               mbar_arrive_expect_tx(bar_kv_full(s), C::TILE_BYTES);
               const CUtensorMap* tm = which ? &p.tm_v : &p.tm_k;
               for (int kb = 0; kb < C::NBOX; ++kb)
-                tma_load_4d(stage_addr(s) + kb * C::BOX_BYTES, tm, bar_kv_full(s), kb * 64, it.hkv,
+                tma_load_4d(stage_addr(s) + kb * C::BOX_BYTES, tm, bar_kv_full(s), kb * C::BOX_ELEMS, it.hkv,
                             (it.kv0 + j) * C::BN, it.b);
             }
           }
@@ -253,17 +274,21 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
       const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
       auto issue_s = [&](int w, uint32_t qa, int sK) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < D / C::KSTEP; ++k) {
           const uint32_t off = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;
-          mma_ss(tS[w], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(stage_addr(sK) + off, 16, 1024),
-                 C::IDESC_S, k > 0);
+          const uint64_t da = smem_desc_sw128(qa + off, 16, 1024), db = smem_desc_sw128(stage_addr(sK) + off, 16, 1024);
+          if constexpr (F8) mma_ss_f8(tS[w], da, db, C::IDESC_S, k > 0);
+          else mma_ss(tS[w], da, db, C::IDESC_S, k > 0);
         }
       };
+      // P (over S's first columns) times V_j: each MMA takes KSTEP keys, 32
+      // bytes of P per row (8 columns) and KSTEP rows of the V tile.
       auto issue_pv = [&](int w, int sV, bool first) {
 #pragma unroll
-        for (int k = 0; k < C::BN / 16; ++k) {
-          mma_ts(tO[w], tS[w] + k * 8, smem_desc_sw128(stage_addr(sV) + k * 16 * 128, C::BOX_BYTES, 1024), C::IDESC_O,
-                 (!first) || k > 0);
+        for (int k = 0; k < C::BN / C::KSTEP; ++k) {
+          const uint64_t db = smem_desc_sw128(stage_addr(sV) + k * C::KSTEP * 128, C::BOX_BYTES, 1024);
+          if constexpr (F8) mma_ts_f8(tO[w], tS[w] + k * 8, db, C::IDESC_O, (!first) || k > 0);
+          else mma_ts(tO[w], tS[w] + k * 8, db, C::IDESC_O, (!first) || k > 0);
         }
       };
       bool ok = true;
@@ -276,9 +301,15 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
         const uint32_t tP[2] = {tmem + C::TM_P, tmem + C::TM_P + 64};
         auto issue_pv_p = [&](int w, int sV, bool first) {
 #pragma unroll
-          for (int k = 0; k < C::BN / 16; ++k) {
-            mma_ts(tO[w], tP[w] + k * 8, smem_desc_sw128(stage_addr(sV) + k * 16 * 128, C::BOX_BYTES, 1024),
-                   C::IDESC_O, (!first) || k > 0);
+          for (int k = 0; k < C::BN / C::KSTEP; ++k) {
+            const uint64_t db = smem_desc_sw128(stage_addr(sV) + k * C::KSTEP * 128, C::BOX_BYTES, 1024);
+            if constexpr (F8) {
+              // P_w in shared memory: K-major, 128-byte rows, 128-byte swizzle
+              const uint64_t da = smem_desc_sw128(sbase + C::OFF_P + w * C::P_BYTES + k * 32, 16, 1024);
+              mma_ss_f8(tO[w], da, db, C::IDESC_O, (!first) || k > 0);
+            } else {
+              mma_ts(tO[w], tP[w] + k * 8, db, C::IDESC_O, (!first) || k > 0);
+            }
           }
         };
         for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -451,7 +482,13 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
             if (2 * c + 1 >= nvalid || 2 * c + 1 < nlo) pr.y = 0.f;
           }
           acc[c & 3] = __fadd2_rn(acc[c & 3], pr);
-          su[c] = pack_bf16x2(pr.x, pr.y);
+          if constexpr (F8) {
+            // four E4M3 values per column; su[c >> 1] was consumed at step c >> 2
+            const uint32_t h = pack_e4m3x2(pr.x, pr.y);
+            su[c >> 1] = (c & 1) ? (su[c >> 1] | (h << 16)) : h;
+          } else {
+            su[c] = pack_bf16x2(pr.x, pr.y);
+          }
         }
         const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
         l += a.x + a.y;
@@ -462,11 +499,22 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
             if (!ok) break;
           }
           tc_fence_after();
-          tmem_st32(tP, su);
-          tmem_st32(tP + 32, su + 32);
+          if constexpr (F8) {
+            // row r of P_w: eight 16-byte chunks, chunk c stored at c ^ (r & 7)
+            // (the 128-byte swizzle the MMA's descriptor names)
+            uint8_t* prow = smem + C::OFF_P + w * C::P_BYTES + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+                  make_uint4(su[4 * c], su[4 * c + 1], su[4 * c + 2], su[4 * c + 3]);
+            fence_proxy_async_smem();
+          } else {
+            tmem_st32(tP, su);
+            tmem_st32(tP + 32, su + 32);
+          }
         } else {
           tmem_st32(tS, su);
-          tmem_st32(tS + 32, su + 32);
+          if constexpr (!F8) tmem_st32(tS + 32, su + 32);
         }
         if (j > 0 && __any_sync(0xffffffffu, move)) {
           // O row *= alpha.  The PV of the previous tile has completed (with
@@ -495,7 +543,7 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
         tc_fence_after();
       }
       const bool in_range = row < p.Tq;
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv_l = (l > 0.f) ? p.o_scale / l : 0.f;
       __nv_bfloat16* orow = p.o + (((size_t)it.b * p.Tq + (in_range ? row : 0)) * p.Hq + it.h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

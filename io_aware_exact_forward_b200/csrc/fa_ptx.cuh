@@ -190,6 +190,29 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// kind::f8f6f4 forms of the two MMAs above (8-bit A and B of the formats the
+// instruction descriptor names; K = 32 elements, 32 bytes, per instruction).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// A from tensor memory: four 8-bit values per 32-bit column, K-major.
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -292,6 +315,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | ((uint32_t)(M >> 4) << 24);          // M / 16
 }
 
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (format code 0)
+// and fp32 accumulation; a_mn / b_mn as above (MN-major is allowed for the
+// 8-bit formats E4M3 and E5M2).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                              // D format: f32
+         | (0u << 7)                            // A format: E4M3
+         | (0u << 10)                           // B format: E4M3
+         | ((uint32_t)a_mn << 15)
+         | ((uint32_t)b_mn << 16)
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------------------
 // Small math helpers
 // ---------------------------------------------------------------------------
@@ -325,6 +361,14 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   // multiplies by 2^n (the magic's own bits vanish in the shift)
   return make_float2(__int_as_float(__float_as_int(p.x) + (int)((uint32_t)__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(p.y) + (int)((uint32_t)__float_as_int(t.y) << 23)));
+}
+
+// Two floats to two E4M3 bytes (round to nearest even, saturating to +-448),
+// `lo` in bits 0-7 and `hi` in bits 8-15.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -141,3 +141,14 @@ def test_context_parallel_decode_argument_checks():
     # O stride not a multiple of 4 floats, or a misaligned O block
     assert lib.fa_decode_merge(al, rows * d + 2, al, rows, al, al, 2, 2, 4, d, NULL) == 3
     assert lib.fa_decode_merge(ctypes.c_void_p(base + 8), rows * d, al, rows, al, al, 2, 2, 4, d, NULL) == 3
+
+
+def test_fp8_forward_argument_checks():
+    lib = fa.load_library()
+    args = (1, 1, 1, 16, 16)
+    # (q, k, v, q_descale, k_descale, v_descale, o, lse, B, Hq, Hkv, Tq, Tk, d, scale, causal, stream)
+    for bad in ((0.0, 1.0, 1.0), (1.0, -1.0, 1.0), (1.0, 1.0, float("inf")), (float("nan"), 1.0, 1.0)):
+        assert lib.fa_forward_fp8(NULL, NULL, NULL, *bad, NULL, NULL, *args, 128, 1.0, 0, NULL) == 1
+    assert lib.fa_forward_fp8(NULL, NULL, NULL, 1.0, 1.0, 1.0, NULL, NULL, *args, 64, 1.0, 0, NULL) == 2
+    assert lib.fa_forward_fp8(NULL, NULL, NULL, 1.0, 1.0, 1.0, NULL, NULL, *args, 128, 1.0, 0, NULL) == 1
+    assert lib.fa_forward_fp8(NULL, NULL, NULL, 1.0, 1.0, 1.0, NULL, NULL, 1, 1, 1, 0, 16, 128, 1.0, 0, NULL) == 0

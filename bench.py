@@ -102,12 +102,20 @@ def load_peaks():
         return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": "fa_fwd.cuh",
+    "fa_bwd_dkdv_kernel": "fa_bwd.cuh",
+    "fa_decode_split_kernel": "fa_decode.cuh",
+}
+
+
+def kernel_source_hash(kernel):
+    """Hash of the source file that holds a kernel's code (the shared PTX
+    wrappers only gain functions, so a kernel's file is what changes it)."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "io_aware_exact_forward_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+    f = KERNEL_SOURCES[kernel]
+    with open(os.path.join(ROOT, "io_aware_exact_forward_b200", "csrc", f), "rb") as fh:
+        h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -119,7 +127,7 @@ def traffic_from_profile(kernel, workload):
         with open(path) as f:
             data = json.load(f)
         ent = data[kernel][workload]
-        if ent.get("source_hash") == kernel_source_hash():
+        if ent.get("source_hash") == kernel_source_hash(kernel):
             return ent["dram_bytes_per_launch"]
     except Exception:
         pass

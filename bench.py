@@ -303,9 +303,60 @@ def run_reference_decode(args, w):
     return 0
 
 
+def run_reference_fp8(args, w):
+    """The oracle's forward on E4M3 inputs on the host cores: each step 256
+    query rows of one head (heads and row blocks cycling over the workload),
+    decoding that head's codes included."""
+    import numpy as np
+    import torch
+    import oracle
+    from workloads import prefill_inputs_e4m3
+    inp = prefill_inputs_e4m3(w.with_(B=1), device="cpu")
+    codes = {n: inp[n].view(torch.uint8).numpy() for n in ("q", "k", "v")}
+    G = w.Hq // w.Hkv
+    T, n_blk = w.T, (w.T + 255) // 256
+
+    def one(s):
+        h, blk = s % w.Hq, (s * 7919) % n_blk
+        rows = np.arange(blk * 256, min(T, blk * 256 + 256))
+        t0 = time.perf_counter()
+        q = oracle.e4m3_decode(codes["q"][0, :, h]) * inp["q_descale"]
+        k = oracle.e4m3_decode(codes["k"][0, :, h // G]) * inp["k_descale"]
+        v = oracle.e4m3_decode(codes["v"][0, :, h // G]) * inp["v_descale"]
+        oracle.head_forward(q, k, v, w.scale, w.causal, rows=rows)
+        dt = time.perf_counter() - t0
+        keys = np.minimum(rows + 1, T).sum() if w.causal else len(rows) * T
+        return dt, 4.0 * w.d * float(keys)
+
+    for s in range(args.warmup):
+        one(s)
+    tot_t, tot_f = 0.0, 0.0
+    for s in range(args.steps):
+        dt, fl = one(s)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": "attention forward TFLOPS (E4M3 inputs, 1xB200) and % of dense E4M3 tensor peak",
+        "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d, "causal": w.causal,
+                   "inputs": "E4M3 codes, per-tensor amax/448 factors",
+                   "step": "256 query rows of one head, forward, codes decoded"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"256 query rows of one head of {w.name} per step, float64 numpy"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return 0
+    if args.fp8:
+        return run_reference_fp8(args, w)
     if w.decode:
         return run_reference_decode(args, w)
     from workloads import prefill_inputs
@@ -957,14 +1008,14 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     dist = None
-    if args.impl == "reference":
-        return run_reference(args, w, rank)
     if args.fp8 and (w.decode or w.d != 128 or w.window):
         print("--fp8 applies to the d = 128 prefill workloads without a window", file=sys.stderr)
         return 2
     if args.cp and (not w.decode or w.window):
         print("--cp applies to the decode workload without a window", file=sys.stderr)
         return 2
+    if args.impl == "reference":
+        return run_reference(args, w, rank)
     if world > 1 or args.cp:
         import datetime
         import torch

@@ -26,8 +26,9 @@
  *       k, v, dk, dv   : [B, Tk, Hkv, d]
  *       lse            : [B, Hq, Tq]   (natural-log units of the scaled scores)
  *   - d must be 64 or 128; Hq % Hkv == 0; B * Hq <= 65535 for the prefill
- *     entry points.  Query head h reads KV head h / (Hq / Hkv) (contiguous
- *     groups).
+ *     entry points and B * Hq <= 2^26 for the decode ones (larger sizes are
+ *     FA_ERR_INVALID_ARG).  Query head h reads KV head h / (Hq / Hkv)
+ *     (contiguous groups).
  *   - Causal rule: key j is visible to query i iff j <= i + (Tk - Tq)
  *     (bottom-right aligned; for Tq == Tk this is j <= i).  A row that sees
  *     no key gets O = 0, LSE = -inf and zero gradients.

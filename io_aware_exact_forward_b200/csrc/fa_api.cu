@@ -482,7 +482,9 @@ static int decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
   if (chunk < 64 || chunk % 64 != 0 || chunk * G > 4096) return FA_ERR_INVALID_ARG;
-  if ((int64_t)Tk_max > (1 << 30) || (int64_t)B * Hq > (1 << 30)) return FA_ERR_INVALID_ARG;
+  // one warp per (sequence, head) row in the merge kernels: 32 * B * Hq
+  // threads must stay below 2^31
+  if ((int64_t)Tk_max > (1 << 30) || (int64_t)B * Hq > (1 << 26)) return FA_ERR_INVALID_ARG;
   if (B == 0) return FA_OK;
   if (!q || !seqlens_k || (!o == !o32) || !lse || (Tk_max > 0 && (!k_cache || !v_cache)))
     return FA_ERR_INVALID_ARG;
@@ -565,7 +567,7 @@ int fa_decode_splitkv_partial(const void* q, const void* k_cache, const void* v_
 
 int fa_decode_merge(const float* o_parts, size_t o_stride, const float* lse_parts, size_t lse_stride, void* o,
                     float* lse, int R, int B, int Hq, int d, void* stream) {
-  if (R < 1 || R > (1 << 20) || B < 0 || Hq < 1 || (int64_t)B * Hq > (1 << 30)) return FA_ERR_INVALID_ARG;
+  if (R < 1 || R > (1 << 20) || B < 0 || Hq < 1 || (int64_t)B * Hq > (1 << 26)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const size_t rows = (size_t)B * Hq;
   if (rows == 0) return FA_OK;

@@ -152,3 +152,12 @@ def test_fp8_forward_argument_checks():
     assert lib.fa_forward_fp8(NULL, NULL, NULL, 1.0, 1.0, 1.0, NULL, NULL, *args, 64, 1.0, 0, NULL) == 2
     assert lib.fa_forward_fp8(NULL, NULL, NULL, 1.0, 1.0, 1.0, NULL, NULL, *args, 128, 1.0, 0, NULL) == 1
     assert lib.fa_forward_fp8(NULL, NULL, NULL, 1.0, 1.0, 1.0, NULL, NULL, 1, 1, 1, 0, 16, 128, 1.0, 0, NULL) == 0
+
+
+def test_decode_row_limit():
+    """One warp per (sequence, head) row in the merge kernels: B * Hq above
+    2^26 is rejected on the host."""
+    lib = fa.load_library()
+    big = (1 << 26) // 32 + 1
+    assert lib.fa_decode_splitkv(*([NULL] * 6), NULL, 0, big, 32, 8, 1024, 128, 0.1, 256, NULL) == 1
+    assert lib.fa_decode_merge(NULL, 0, NULL, 0, NULL, NULL, 2, big, 32, 128, NULL) == 1

@@ -283,6 +283,8 @@ def decode_merge(o_parts, lse_parts, out=None, lse=None):
     any stride along R (e.g. views into one packed all-gather buffer) but must
     be contiguous within a partial.  Returns O bf16 [B,Hq,d], LSE [B,Hq]."""
     lib = load_library()
+    if o_parts.dim() != 4 or o_parts.shape[0] < 1:
+        raise ValueError(f"o_parts must be [R >= 1, B, Hq, d], got {tuple(o_parts.shape)}")
     R, B, Hq, d = o_parts.shape
     dev = o_parts.device
     for n, t in (("o_parts", o_parts), ("lse_parts", lse_parts)):

@@ -54,6 +54,8 @@ def parse_args():
                     help="sliding window of that many keys (prefill: implies causal; decode: last keys)")
     ap.add_argument("--fp8", action="store_true",
                     help="prefill, d = 128 only: the E4M3 forward (fa_forward_fp8) alone")
+    ap.add_argument("--dropout", type=float, default=None,
+                    help="prefill: the forward with fused dropout of this rate alone (fa_forward_dropout)")
     ap.add_argument("--cp", action="store_true",
                     help="decode only: context-parallel, every sequence's cache cut into one share per GPU")
     ap.add_argument("--batch", type=int, default=None,
@@ -352,11 +354,51 @@ def run_reference_fp8(args, w):
     return 0
 
 
+def run_reference_dropout(args, w):
+    """The oracle's forward with dropout on P on the host cores: each step
+    one (batch, head) of the workload (heads cycling)."""
+    import oracle
+    from oracle import dropout as dr
+    from workloads import prefill_inputs, to_f64
+    inp = prefill_inputs(w.with_(B=1), device="cpu")
+    G = w.Hq // w.Hkv
+    f_fwd, _ = flops(w)
+    per_head = f_fwd / (w.B * w.Hq)
+
+    def one(s):
+        h = s % w.Hq
+        t0 = time.perf_counter()
+        dr.head_forward_dropout(to_f64(inp["q"][0, :, h]), to_f64(inp["k"][0, :, h // G]),
+                                to_f64(inp["v"][0, :, h // G]), w.scale, w.causal, args.dropout, 0x5EED0000, s, h)
+        return time.perf_counter() - t0
+
+    for s in range(args.warmup):
+        one(s)
+    tot = sum(one(s) for s in range(args.steps))
+    value = per_head * args.steps / tot / 1e12
+    line = {
+        "impl": "reference",
+        "metric": "attention forward TFLOPS with fused dropout (bf16, 1xB200) and % of dense tensor peak",
+        "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d, "causal": w.causal,
+                   "dropout": args.dropout, "step": "one (batch, head) of the workload, forward with dropout"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one (batch, head) of {w.name} per step, float64 numpy"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return 0
     if args.fp8:
         return run_reference_fp8(args, w)
+    if args.dropout is not None:
+        return run_reference_dropout(args, w)
     if w.decode:
         return run_reference_decode(args, w)
     from workloads import prefill_inputs
@@ -868,6 +910,92 @@ def run_fp8_forward(args, w, rank, world, dist):
     return 0
 
 
+def run_dropout_forward(args, w, rank, world, dist):
+    """The forward with fused dropout on P (rate args.dropout) on a prefill
+    workload: one step is one fa_forward_dropout launch (inputs resident, L2
+    flushed between launches).  value is algorithmic TFLOP/s (4 B Hq d
+    pairs, the dropout's mask work not counted); the plain forward is timed
+    the same way in the same run for the overhead."""
+    import ctypes
+    import torch
+    import io_aware_exact_forward_b200 as fa
+    from workloads import prefill_inputs
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = fa.load_library()
+    inp = prefill_inputs(w, device=dev, seed=w.seed + rank)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    P = ctypes.c_void_p
+    stream = torch.cuda.current_stream(dev)
+    sp = P(stream.cuda_stream)
+    base = (P(q.data_ptr()), P(k.data_ptr()), P(v.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
+            B, Hq, Hkv, T, T, d, w.scale, int(w.causal))
+    seed = 0x5EED0000 + rank
+
+    def step(s_, drop=True):
+        st = (lib.fa_forward_dropout(*base, float(args.dropout), seed, s_, sp) if drop
+              else lib.fa_forward(*base, sp))
+        if st != 0:
+            raise RuntimeError(f"forward: {fa.STATUS.get(st, st)}")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(drop):
+        for s_ in range(args.warmup):
+            step(s_, drop)
+        barrier()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for s_ in range(args.steps):
+            flush.fill_(s_ & 0xFF)
+            evs[s_][0].record(stream)
+            step(s_, drop)       # a new offset every step: a new mask
+            evs[s_][1].record(stream)
+        barrier()
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), dist, dev)
+
+    with ClockSampler(local) as clocks:
+        ms = timed(True)
+    ms_plain = timed(False)
+    if lib.fa_check(sp) != 0:
+        raise RuntimeError("device status set during the timed region")
+    f_fwd, _ = flops(w)
+    value = job_rate(f_fwd, world, args.steps, ms) / 1e12
+    peaks = load_peaks()
+    if rank == 0:
+        line = {
+            "metric": "attention forward TFLOPS with fused dropout (bf16, 1xB200) and % of dense tensor peak",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
+                       "dropout": args.dropout, "l2": "256 MiB flush between launches", "seed": w.seed},
+            "plain_forward": {"ms_per_step": ms_plain / args.steps,
+                              "tflops": job_rate(f_fwd, world, args.steps, ms_plain) / 1e12},
+            "roofline": {"kernel": "fa_fwd_kernel<d, false, true>", "bound": "tensor", "achieved": value / world,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": value / world / peaks["bf16_tflops"],
+                         "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": None,
+                         "algorithmic_per_launch": f_fwd},
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+            "cpu_baseline": None,
+            "e2e": None,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_decode_cp(args, w, rank, world, dist):
     """Context-parallel decode of the same batch: every sequence's cache is
     cut into `world` contiguous shares and rank r holds share r.  One step is
@@ -1011,6 +1139,10 @@ def main():
     if args.fp8 and (w.decode or w.d != 128 or w.window):
         print("--fp8 applies to the d = 128 prefill workloads without a window", file=sys.stderr)
         return 2
+    if args.dropout is not None and (w.decode or w.window or not (0.0 <= args.dropout < 1.0)):
+        print("--dropout takes a rate in [0, 1) and applies to the prefill workloads without a window",
+              file=sys.stderr)
+        return 2
     if args.cp and (not w.decode or w.window):
         print("--cp applies to the decode workload without a window", file=sys.stderr)
         return 2
@@ -1029,6 +1161,8 @@ def main():
     try:
         if args.fp8:
             return run_fp8_forward(args, w, rank, world, dist)
+        if args.dropout is not None:
+            return run_dropout_forward(args, w, rank, world, dist)
         if w.decode and args.cp:
             return run_decode_cp(args, w, rank, world, dist)
         if w.decode:

@@ -100,6 +100,25 @@ int fa_forward_window(const void* q, const void* k, const void* v, void* o, floa
                       void* stream);
 
 /*
+ * fa_forward_dropout -- fa_forward with dropout on P fused into the kernel
+ * ("Efficient attention: memory-bound", "Real code moves even more", lists
+ * dropout among the elementwise steps on P before the final product):
+ *   O = (P * Z) V / (t / 256),  LSE that of the undropped P,
+ * where Z_ij keeps (i, j) with probability t / 256, t = round(256 (1 - p_drop))
+ * clamped to 1..256 (p_drop is used to the nearest 1/256).  Z is regenerated
+ * from Philox-4x32-10 (Salmon et al., SC 2011): the block of rows 4a..4a+3 and
+ * keys 4c..4c+3 of head h of batch b uses counter (a, c, b * Hq + h, offset)
+ * and key (seed mod 2^32, seed >> 32); word w of its output is row 4a + w and
+ * byte j of that word key 4c + j, kept iff the byte < t.  The same (seed,
+ * offset) always gives the same mask.
+ *   p_drop in [0, 1) (else FA_ERR_INVALID_ARG); p_drop = 0 gives fa_forward.
+ *   Other arguments and errors as fa_forward.  bf16 only; no window.
+ */
+int fa_forward_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                       int Hkv, int Tq, int Tk, int d, float scale, int causal, float p_drop,
+                       unsigned long long seed, unsigned int offset, void* stream);
+
+/*
  * fa_forward_fp8 -- fa_forward with 8-bit inputs: the low-precision forward
  * that "FlashAttention" (interview track, "In practice") lists for FA3, here
  * on B200's kind::f8f6f4 tensor-core MMAs.

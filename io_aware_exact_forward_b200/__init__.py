@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     decode_splitkv_partial,
     decode_workspace_bytes,
     forward,
+    forward_dropout,
     forward_fp8,
     load_library,
     selftest_bounded_wait,

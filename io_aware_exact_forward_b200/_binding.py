@@ -33,6 +33,8 @@ SIGNATURES = {
     "fa_version": (_c_int, []),
     "fa_forward": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_forward_window": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_forward_dropout": (_c_int, [_vp] * 5 + [_c_int] * 6 + [_c_float, _c_int, _c_float, ctypes.c_ulonglong,
+                                                               ctypes.c_uint, _vp]),
     "fa_forward_fp8": (_c_int, [_vp] * 3 + [_c_float] * 3 + [_vp, _vp] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_workspace_bytes": (_c_size, [_c_int] * 6),
     "fa_backward": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
@@ -132,6 +134,32 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, window=None):
         st = lib.fa_forward_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tk, d,
                                    float(scale), int(window), _stream_ptr(dev))
         _raise("fa_forward_window", st)
+    return out, lse
+
+
+def forward_dropout(q, k, v, p_drop, seed, offset=0, scale=None, causal=False, out=None, lse=None):
+    """O, LSE of attention with dropout on P (fa_forward_dropout): each
+    probability kept with probability round(256 (1 - p_drop)) / 256 by a
+    Philox-4x32-10 mask regenerated from (seed, offset), the kept ones scaled
+    up by the inverse.  bf16 tensors as in forward()."""
+    lib = load_library()
+    B, Tq, Hq, d = q.shape
+    Tk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_dev(n, t, torch.bfloat16, dev)
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=dev)
+    _check_dev("out", out, torch.bfloat16, dev)
+    _check_dev("lse", lse, torch.float32, dev)
+    st = lib.fa_forward_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tk, d,
+                                float(scale), int(bool(causal)), float(p_drop), int(seed) & (2 ** 64 - 1),
+                                int(offset) & 0xFFFFFFFF, _stream_ptr(dev))
+    _raise("fa_forward_dropout", st)
     return out, lse
 
 

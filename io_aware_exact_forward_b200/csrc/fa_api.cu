@@ -126,6 +126,8 @@ static int device_setup_impl() {
   if (!st) st = set_smem(fa_fwd_kernel<64>, FwdCfg<64>::SMEM_BYTES);
   if (!st) st = set_smem(fa_fwd_kernel<128>, FwdCfg<128>::SMEM_BYTES);
   if (!st) st = set_smem(fa_fwd_kernel<128, true>, FwdCfg<128, true>::SMEM_BYTES);
+  if (!st) st = set_smem(fa_fwd_kernel<64, false, true>, FwdCfg<64>::SMEM_BYTES);
+  if (!st) st = set_smem(fa_fwd_kernel<128, false, true>, FwdCfg<128>::SMEM_BYTES);
   if (!st) st = bwd_setup();
   if (!st) st = decode_setup();
   return st;
@@ -205,10 +207,14 @@ int fa_version(void) { return 100; }
 
 // window > 0: sliding window of that many keys (the caller passes causal = 1).
 // f8: q, k, v are E4M3; `qk_factor` multiplies the scores' scale and
-// `o_scale` the output (the dequantising factors).
+// `o_scale` the output (the dequantising factors).  drop_t in 1..255: dropout
+// on P with keep threshold drop_t (o_scale is then 256 / drop_t), Philox key
+// (seed_lo, seed_hi) and counter word `drop_offset`.
 static int forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                         int Hkv, int Tq, int Tk, int d, float scale, int causal, int window, void* stream,
-                        bool f8 = false, float qk_factor = 1.f, float o_scale = 1.f) {
+                        bool f8 = false, float qk_factor = 1.f, float o_scale = 1.f, uint32_t drop_t = 256,
+                        uint32_t seed_lo = 0, uint32_t seed_hi = 0, uint32_t drop_offset = 0) {
+  const bool drop = drop_t < 256;
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
   if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
@@ -233,6 +239,10 @@ static int forward_impl(const void* q, const void* k, const void* v, void* o, fl
   p.window = window;
   p.scale_log2 = scale * qk_factor * 1.4426950408889634f;
   p.o_scale = o_scale;
+  p.drop_t = drop_t;
+  p.seed_lo = seed_lo;
+  p.seed_hi = seed_hi;
+  p.drop_offset = drop_offset;
   p.n_mblocks = (Tq + 255) / 256;
   p.n_items = B * Hq * p.n_mblocks;
   p.wait_limit_ns = kWaitLimitNs;
@@ -245,6 +255,10 @@ static int forward_impl(const void* q, const void* k, const void* v, void* o, fl
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (f8)
     fa_fwd_kernel<128, true><<<grid, FwdCfg<128, true>::THREADS, FwdCfg<128, true>::SMEM_BYTES, s>>>(p);
+  else if (drop && d == 64)
+    fa_fwd_kernel<64, false, true><<<grid, FwdCfg<64>::THREADS, FwdCfg<64>::SMEM_BYTES, s>>>(p);
+  else if (drop)
+    fa_fwd_kernel<128, false, true><<<grid, FwdCfg<128>::THREADS, FwdCfg<128>::SMEM_BYTES, s>>>(p);
   else if (d == 64)
     fa_fwd_kernel<64><<<grid, FwdCfg<64>::THREADS, FwdCfg<64>::SMEM_BYTES, s>>>(p);
   else
@@ -263,6 +277,17 @@ int fa_forward_window(const void* q, const void* k, const void* v, void* o, floa
                       int Hkv, int Tq, int Tk, int d, float scale, int window, void* stream) {
   if (window < 1) return FA_ERR_INVALID_ARG;
   return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, d, scale, 1, window, stream);
+}
+
+int fa_forward_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                       int Hkv, int Tq, int Tk, int d, float scale, int causal, float p_drop,
+                       unsigned long long seed, unsigned int offset, void* stream) {
+  if (!(p_drop >= 0.f && p_drop < 1.f)) return FA_ERR_INVALID_ARG;
+  long t = lrintf(256.f * (1.f - p_drop));
+  t = t < 1 ? 1 : (t > 256 ? 256 : t);
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0, stream, false, 1.f,
+                      256.f / (float)t, (uint32_t)t, (uint32_t)(seed & 0xFFFFFFFFull), (uint32_t)(seed >> 32),
+                      offset);
 }
 
 int fa_forward_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,

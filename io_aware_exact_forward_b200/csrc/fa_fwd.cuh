@@ -40,6 +40,12 @@
 // unrounded fp32 p.  P goes to shared memory (16 KB per query tile), so that
 // the next S overlaps the softmax as in the d = 64 kernel.
 //
+// Dropout variant (DROP = true, bf16): P is multiplied by a keep mask before
+// P V ("Efficient attention: memory-bound", "Real code moves even more", puts
+// dropout on the probabilities before the final product); the mask is
+// regenerated from Philox-4x32-10 for each tile, l sums the undropped P, and
+// the epilogue scales O by 256 / t.
+//
 // The rescale is lazy: a row keeps its reference maximum until the running
 // maximum exceeds it by more than 8 (log2 units), so exponentials stay below
 // 2^8.  l and u always share one reference, so the result is the same
@@ -60,7 +66,9 @@ struct FwdParams {
   int causal;
   int window;         // > 0: sliding window of that many keys (implies causal)
   float scale_log2;   // scale * log2(e) (times the q and k factors for E4M3 inputs)
-  float o_scale;      // multiplies O = u / l: 1, or the v factor for E4M3 inputs
+  float o_scale;      // multiplies O = u / l: 1, the v factor for E4M3 inputs, or 256 / t with dropout
+  uint32_t drop_t;    // dropout: keep iff the Philox byte < drop_t (1..255)
+  uint32_t seed_lo, seed_hi, drop_offset;  // dropout: Philox key and counter word 3
   int n_mblocks;      // ceil(Tq / 256): work items per (batch, head)
   int n_items;        // B * Hq * n_mblocks
   unsigned long long wait_limit_ns;
@@ -148,7 +156,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
   return it;
 }
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool DROP = false>
 __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
@@ -427,6 +435,11 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
       float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
       float l = 0.f;
       for (int j = 0; j < it.n_kv; ++j) {
+        // dropout: this tile's keep bits, made while the tensor core computes S
+        uint32_t keep[4];
+        if constexpr (DROP)
+          dropout_keep_128(keep, row, (it.kv0 + j) * C::BN, (uint32_t)(it.b * p.Hq + it.h), p.drop_offset,
+                           p.seed_lo, p.seed_hi, p.drop_t);
         ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(w), (g + j) & 1, wc));
         if (!ok) break;
         tc_fence_after();
@@ -481,7 +494,12 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
             if (2 * c >= nvalid || 2 * c < nlo) pr.x = 0.f;
             if (2 * c + 1 >= nvalid || 2 * c + 1 < nlo) pr.y = 0.f;
           }
-          acc[c & 3] = __fadd2_rn(acc[c & 3], pr);
+          acc[c & 3] = __fadd2_rn(acc[c & 3], pr);   // l sums the undropped p
+          if constexpr (DROP) {
+            const uint32_t kb = keep[c >> 4] >> ((2 * c) & 31);
+            pr.x = (kb & 1u) ? pr.x : 0.f;
+            pr.y = (kb & 2u) ? pr.y : 0.f;
+          }
           if constexpr (F8) {
             // four E4M3 values per column; su[c >> 1] was consumed at step c >> 2
             const uint32_t h = pack_e4m3x2(pr.x, pr.y);

@@ -363,6 +363,61 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (int)((uint32_t)__float_as_int(t.y) << 23)));
 }
 
+// ---------------------------------------------------------------------------
+// Dropout mask: Philox-4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel
+// random numbers: as easy as 1, 2, 3", SC 2011), one block per 4 x 4 block of
+// (query, key) pairs
+// ---------------------------------------------------------------------------
+
+// Ten rounds: multiply words 0 and 2 by the round constants into (hi, lo)
+// pairs, mix with words 1 and 3 and the key, bump the key by the Weyl
+// increments between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+  constexpr uint32_t kM0 = 0xD2511F53u, kM1 = 0xCD9E8D57u, kW0 = 0x9E3779B9u, kW1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += kW0;
+      k1 += kW1;
+    }
+    const uint32_t hi0 = __umulhi(kM0, c.x), lo0 = kM0 * c.x;
+    const uint32_t hi1 = __umulhi(kM1, c.z), lo1 = kM1 * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// Keep bits of query row `row` for the 128 keys key0 .. key0 + 127 (key0 a
+// multiple of 16): bit k of mask[k >> 5] is key key0 + k.  The block of rows
+// 4a..4a+3 and keys 4c..4c+3 is Philox at counter (a, c, bh, offset); its
+// word w is row 4a + w, byte j of that word key 4c + j, kept iff the byte is
+// below t (1 <= t <= 255).  The four lanes of a quad hold rows 4a..4a+3 (row
+// & 3 == lane & 3) and share blocks: lane q computes key groups 4m + q and
+// passes each quad-mate its row's word.
+__device__ __forceinline__ void dropout_keep_128(uint32_t (&mask)[4], int row, int key0, uint32_t bh,
+                                                 uint32_t offset, uint32_t k0, uint32_t k1, uint32_t t) {
+  const int lane = threadIdx.x & 31;
+  const int q = lane & 3;
+  const uint32_t tt = t * 0x01010101u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mask[i] = 0u;
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const uint4 wv = philox4x32_10(make_uint4((uint32_t)row >> 2, (uint32_t)(key0 >> 2) + 4 * m + q, bh, offset), k0, k1);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int src = (q + s) & 3;       // lane of the quad whose block this is
+      const int want = (q - s) & 3;      // the word the receiving lane needs
+      const uint32_t send = want == 0 ? wv.x : want == 1 ? wv.y : want == 2 ? wv.z : wv.w;
+      const uint32_t got = s == 0 ? send : __shfl_sync(0xffffffffu, send, (lane & ~3) | src);
+      const uint32_t lt = __vcmpltu4(got, tt);   // 0xFF in each byte below t
+      const uint32_t bits = ((lt >> 7) & 1u) | ((lt >> 14) & 2u) | ((lt >> 21) & 4u) | ((lt >> 28) & 8u);
+      // keys 4 * (4m + src) .. + 3 of the tile: word m / 2, bits 16 (m & 1) + 4 src
+      mask[m >> 1] |= bits << (16 * (m & 1) + 4 * src);
+    }
+  }
+}
+
 // Two floats to two E4M3 bytes (round to nearest even, saturating to +-448),
 // `lo` in bits 0-7 and `hi` in bits 8-15.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {

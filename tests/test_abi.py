@@ -161,3 +161,13 @@ def test_decode_row_limit():
     big = (1 << 26) // 32 + 1
     assert lib.fa_decode_splitkv(*([NULL] * 6), NULL, 0, big, 32, 8, 1024, 128, 0.1, 256, NULL) == 1
     assert lib.fa_decode_merge(NULL, 0, NULL, 0, NULL, NULL, 2, big, 32, 128, NULL) == 1
+
+
+def test_dropout_forward_argument_checks():
+    lib = fa.load_library()
+    args = (1, 1, 1, 16, 16, 64, 1.0, 0)
+    for p in (-0.1, 1.0, 1.5, float("nan")):
+        assert lib.fa_forward_dropout(NULL, NULL, NULL, NULL, NULL, *args, p, 1, 0, NULL) == 1
+    assert lib.fa_forward_dropout(NULL, NULL, NULL, NULL, NULL, *args, 0.1, 1, 0, NULL) == 1   # null pointers
+    assert lib.fa_forward_dropout(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 16, 16, 96, 1.0, 0, 0.1, 1, 0,
+                                  NULL) == 2

@@ -1,0 +1,59 @@
+"""Fused-dropout forward parity: fa_forward_dropout against the float64
+oracle's attention with dropout on P (oracle.dropout), which draws the same
+Philox-4x32-10 mask from the same (seed, offset).  The keep decisions are
+integer and must agree exactly, so O agrees to the bf16 path's tolerances
+(compared after undoing the 256/t scale, which both sides apply); LSE is
+that of the undropped P."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import dropout as dr
+from workloads import WORKLOADS, prefill_inputs, to_f64
+from _parity import assert_lse_close, assert_o_close
+
+pytestmark = pytest.mark.gpu
+
+fa = pytest.importorskip("io_aware_exact_forward_b200")
+
+CASES = [
+    # B, Hq, Hkv, Tq, Tk, d, causal, p
+    (1, 2, 2, 300, 300, 64, False, 0.1),
+    (1, 2, 1, 517, 517, 128, True, 0.5),
+    (2, 4, 2, 200, 450, 64, True, 0.3),
+    (1, 2, 2, 450, 200, 128, True, 0.2),     # early rows see no key
+    (1, 8, 1, 256, 256, 64, False, 0.9),     # G = 8, heavy dropout
+    (1, 1, 1, 2048, 2048, 64, False, 0.25),  # long rows: many key tiles
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Tq,Tk,d,causal,p", CASES)
+def test_dropout_forward(B, Hq, Hkv, Tq, Tk, d, causal, p):
+    w = WORKLOADS[2].with_(B=B, Hq=Hq, Hkv=Hkv, d=d, causal=causal)
+    inp = prefill_inputs(w, seed=61 + Tq + 3 * Tk + d, Tq=Tq, Tk=Tk)
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    seed, offset = 0x5EED_0000_1234 + Tq, 3 + Hq
+    o, lse = fa.forward_dropout(q, k, v, p, seed, offset, scale=w.scale, causal=causal)
+    assert fa.check() == 0
+    O, LSE = dr.attention_forward_dropout(to_f64(inp["q"]), to_f64(inp["k"]), to_f64(inp["v"]), w.scale, causal,
+                                          p, seed, offset)
+    back = dr.keep_threshold(p) / 256.0
+    assert_o_close(to_f64(o.cpu()) * back, O * back)
+    assert_lse_close(lse.cpu().numpy(), LSE)
+
+
+def test_dropout_zero_rate_is_the_plain_forward_and_masks_repeat():
+    w = WORKLOADS[2].with_(B=1, Hq=2, Hkv=2, d=64, causal=True)
+    inp = prefill_inputs(w, seed=5, Tq=384, Tk=384)
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    o0, l0 = fa.forward(q, k, v, scale=w.scale, causal=True)
+    o1, l1 = fa.forward_dropout(q, k, v, 0.0, 99, 0, scale=w.scale, causal=True)
+    a, la = fa.forward_dropout(q, k, v, 0.4, 99, 0, scale=w.scale, causal=True)
+    b, lb = fa.forward_dropout(q, k, v, 0.4, 99, 0, scale=w.scale, causal=True)
+    c, _ = fa.forward_dropout(q, k, v, 0.4, 99, 1, scale=w.scale, causal=True)
+    assert fa.check() == 0
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+    assert torch.equal(a, b) and torch.equal(la, lb) and torch.equal(la, l0)
+    assert not torch.equal(a, c)

@@ -171,3 +171,41 @@ def test_dropout_forward_argument_checks():
     assert lib.fa_forward_dropout(NULL, NULL, NULL, NULL, NULL, *args, 0.1, 1, 0, NULL) == 1   # null pointers
     assert lib.fa_forward_dropout(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 16, 16, 96, 1.0, 0, 0.1, 1, 0,
                                   NULL) == 2
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/fa.h compiles as strict C99 and a C program links against
+    libfa.so and calls it (host-side checks only, no GPU)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fa.load_library()
+    src = tmp_path / "t.c"
+    src.write_text(
+        '#include "fa.h"\n#include <string.h>\n'
+        "int main(void) {\n"
+        '  if (strcmp(fa_status_string(FA_ERR_ALIGNMENT), "FA_ERR_ALIGNMENT")) return 1;\n'
+        "  if (fa_forward(0, 0, 0, 0, 0, 1, 1, 1, 16, 16, 96, 1.0f, 0, 0) != FA_ERR_UNSUPPORTED) return 2;\n"
+        "  if (fa_decode_workspace_bytes(1, 1, 10, 96, 256) != 0) return 3;\n"
+        "  return fa_version() > 0 ? 0 : 4;\n}\n")
+    libdir = os.path.dirname(fa.LIB_PATH)
+    exe = tmp_path / "t"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lfa", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_new_entry_points_check_alignment_before_launch():
+    lib = fa.load_library()
+    buf = (ctypes.c_uint8 * 256)()
+    base = ctypes.addressof(buf) + (16 - ctypes.addressof(buf) % 16) % 16
+    al, odd = ctypes.c_void_p(base), ctypes.c_void_p(base + 4)
+    # dropout forward, misaligned output
+    assert lib.fa_forward_dropout(al, al, al, odd, al, 1, 1, 1, 16, 16, 64, 1.0, 0, 0.1, 1, 0, NULL) == 3
+    # fp8 forward, misaligned q
+    assert lib.fa_forward_fp8(odd, al, al, 1.0, 1.0, 1.0, al, al, 1, 1, 1, 16, 16, 128, 1.0, 0, NULL) == 3
+    # partial decode, misaligned fp32 output
+    assert lib.fa_decode_splitkv_partial(al, al, al, al, odd, al, al, 1 << 20, 1, 4, 4, 64, 128, 0.1, 256,
+                                         NULL) == 3

@@ -111,3 +111,52 @@ def test_shard_seqlens_contiguous_split():
     assert packed_block_floats(1, 1, 64) == 68 and packed_block_floats(2, 4, 128) == 1032
     with pytest.raises(ValueError):
         shard_seqlens(sl, 0, 0)
+
+
+def _failing_worker(rank, world, port, out):
+    import datetime
+    import time
+
+    import torch.distributed as dist
+
+    from io_aware_exact_forward_b200 import context_parallel as cp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        out.put((rank, "failed before the exchange"))
+        out.close()
+        out.join_thread()        # the message is out before the process ends
+        os._exit(3)              # the rank dies between steps, with nothing in flight
+    inp = _inputs()
+
+    def partial(q, k, v, seqlens, scale, chunk, workspace, out, lse):
+        out.zero_()
+        lse.fill_(float("-inf"))
+
+    t0 = time.monotonic()
+    try:
+        cp._cp_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], SCALE, 256, None, None, partial,
+                      lambda o, l: (o, l))
+        out.put((rank, "no error"))
+    except Exception as e:      # the exchange reports the lost peer instead of hanging
+        out.put((rank, f"error after {time.monotonic() - t0:.1f} s: {type(e).__name__}"))
+
+
+def test_lost_rank_fails_the_exchange_instead_of_hanging():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=90) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    assert res[1] == "failed before the exchange"
+    assert res[0].startswith("error after"), res[0]
+    assert float(res[0].split()[2]) < 60.0
+    assert procs[1].exitcode == 3

@@ -209,3 +209,17 @@ def test_new_entry_points_check_alignment_before_launch():
     # partial decode, misaligned fp32 output
     assert lib.fa_decode_splitkv_partial(al, al, al, al, odd, al, al, 1 << 20, 1, 4, 4, 64, 128, 0.1, 256,
                                          NULL) == 3
+
+
+def test_every_exported_symbol_is_declared():
+    """The library exports no fa_* function that include/fa.h does not
+    declare (so the header is the whole boundary)."""
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("no nm")
+    fa.load_library()
+    out = subprocess.run([nm, "-D", "--defined-only", fa.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines() if ln.split() and ln.split()[-1].startswith("fa_")})
+    assert exported == _header_functions()

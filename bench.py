@@ -49,6 +49,10 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="headline workload only (by default the d=128 prefill and decode workloads are timed too)")
+    ap.add_argument("--extra-steps", type=int, default=30,
+                    help="timed steps of the T=8192 workload in the extra set (T=32768: a third; decode: x10)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--window", type=int, default=None,
                     help="sliding window of that many keys (prefill: implies causal; decode: last keys)")
@@ -294,6 +298,8 @@ def run_reference_decode(args, w):
         "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
+        # a token decodes all Hkv groups of its sequence
+        "tokens_per_s": args.steps / w.Hkv / tot_t,
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Tk_max": w.T, "d": w.d,
                    "chunk": w.chunk, "window": w.window or None,
                    "step": "one (sequence, KV head) group of the workload"},
@@ -343,6 +349,7 @@ def run_reference_fp8(args, w):
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
+        "tokens_per_s": tokens_at_rate(value, flops(w)[0], prefill_tokens(w)),
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d, "causal": w.causal,
                    "inputs": "E4M3 codes, per-tensor amax/448 factors",
                    "step": "256 query rows of one head, forward, codes decoded"},
@@ -382,6 +389,7 @@ def run_reference_dropout(args, w):
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
+        "tokens_per_s": tokens_at_rate(value, f_fwd, prefill_tokens(w)),
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d, "causal": w.causal,
                    "dropout": args.dropout, "step": "one (batch, head) of the workload, forward with dropout"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
@@ -416,6 +424,7 @@ def run_reference(args, w, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "tokens_per_s": tokens_at_rate(value, sum(flops(w)), prefill_tokens(w)),
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d,
                    "causal": w.causal, "window": w.window or None,
                    "step": "one head of the workload, forward + backward"},
@@ -451,68 +460,159 @@ def job_rate(work_per_rank_step, world, steps, elapsed_ms):
 # libfa arm
 # ---------------------------------------------------------------------------
 
+class _PrefillRun:
+    """Device buffers and the four launches of one fwd+bwd step of a prefill
+    workload, called through the C ABI."""
+
+    def __init__(self, lib, fa, w, dev, seed):
+        import ctypes
+        import torch
+        from workloads import prefill_inputs
+        self.fa, self.lib, self.w, self.dev = fa, lib, w, dev
+        inp = prefill_inputs(w, device=dev, seed=seed)
+        self.q, self.k, self.v, self.do = inp["q"], inp["k"], inp["v"], inp["do"]
+        B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+        self.ws_bytes = lib.fa_backward_workspace_bytes(B, Hq, Hkv, T, T, d)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
+        P = ctypes.c_void_p
+        self.pq, self.pk, self.pv, self.pdo, self.po, self.plse = (
+            P(t.data_ptr()) for t in (self.q, self.k, self.v, self.do, self.o, self.lse))
+        self.pdq, self.pdk, self.pdv, self.pws = (P(t.data_ptr()) for t in (self.dq, self.dk, self.dv, self.ws))
+        self.stream = torch.cuda.current_stream(dev)
+        self.sp = P(self.stream.cuda_stream)
+        # with a sliding window the windowed entry points take the window in
+        # place of the causal flag
+        self.fwd_fn, self.dkdv_fn, self.mask_arg = lib.fa_forward, lib.fa_backward_dkdv, int(w.causal)
+        if w.window:
+            self.fwd_fn, self.dkdv_fn, self.mask_arg = lib.fa_forward_window, lib.fa_backward_dkdv_window, w.window
+
+    def _check(self, st, name):
+        if st != 0:
+            raise RuntimeError(f"{name}: {self.fa.STATUS.get(st, st)}")
+
+    def step(self, evs=None):
+        w, lib, s = self.w, self.lib, self.stream
+        B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
+        if evs: evs[0].record(s)
+        self._check(self.fwd_fn(self.pq, self.pk, self.pv, self.po, self.plse, B, Hq, Hkv, T, T, d, w.scale,
+                                self.mask_arg, self.sp), "fa_forward")
+        if evs: evs[1].record(s)
+        self._check(lib.fa_backward_preprocess(self.po, self.plse, self.pdo, self.pws, self.ws_bytes, B, Hq, Hkv, T,
+                                               T, d, self.sp), "preprocess")
+        if evs: evs[2].record(s)
+        self._check(self.dkdv_fn(self.pq, self.pk, self.pv, self.pdo, self.pdk, self.pdv, self.pws, self.ws_bytes,
+                                 B, Hq, Hkv, T, T, d, w.scale, self.mask_arg, self.sp), "dkdv")
+        if evs: evs[3].record(s)
+        self._check(lib.fa_backward_dq_finalize(self.pdq, self.pws, self.ws_bytes, B, Hq, Hkv, T, T, d, self.sp),
+                    "dq_finalize")
+        if evs: evs[4].record(s)
+
+    KERNELS_PER_STEP = 4
+
+    def timed(self, steps, warmup, barrier):
+        """Warm-up, then `steps` timed steps with events around every launch.
+        Returns (elapsed ms of the whole timed region on this rank, average
+        ms of each of the four launches)."""
+        import torch
+        for _ in range(warmup):
+            self.step()
+        barrier()
+        if self.lib.fa_check(self.sp) != 0:
+            raise RuntimeError("device status set during warm-up")
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        t0.record(self.stream)
+        for s_ in range(steps):
+            self.step(evs[s_])
+        t1.record(self.stream)
+        barrier()
+        if self.lib.fa_check(self.sp) != 0:
+            raise RuntimeError("device status set during the timed region")
+        seg = [sum(evs[s_][i].elapsed_time(evs[s_][i + 1]) for s_ in range(steps)) / steps for i in range(4)]
+        return t0.elapsed_time(t1), seg
+
+
+def prefill_tokens(w):
+    """Tokens of one prefill step: B * T."""
+    return w.B * w.T
+
+
+def tokens_at_rate(tflops, flops_per_step, tokens_per_step):
+    """Tokens per second of a run that reaches `tflops` on a workload whose
+    step does `flops_per_step` over `tokens_per_step` tokens."""
+    return tflops * 1e12 * tokens_per_step / flops_per_step
+
+
+def extra_workloads(args, lib, fa, dev, rank, world, dist, barrier):
+    """The long-context prefill workloads and the decode workload, each timed
+    on the device in the same run as the headline workload (fewer steps: a
+    step is 10-40 ms there).  Summaries only; each has its own bench line
+    with `--workload N`."""
+    from workloads import WORKLOADS
+    import torch
+    peaks = load_peaks()
+    out = {}
+    for idx, steps in ((3, args.extra_steps), (4, max(3, args.extra_steps // 3))):
+        w = WORKLOADS[idx]
+        run = _PrefillRun(lib, fa, w, dev, w.seed + rank)
+        elapsed, seg = run.timed(steps, 3, barrier)
+        elapsed = max_over_ranks(elapsed, dist, dev)
+        f_fwd, f_bwd = flops(w)
+        value = job_rate(f_fwd + f_bwd, world, steps, elapsed) / 1e12
+        ms = elapsed / steps
+        out[w.name] = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "ms_per_step": ms, "steps": steps, "warmup": 3,
+            "frac": value / world / peaks["bf16_tflops"],
+            "tokens_per_s": world * prefill_tokens(w) / (ms * 1e-3),
+            "per_kernel_ms": {"fa_fwd_kernel": seg[0], "fa_bwd_preprocess_kernel": seg[1],
+                              "fa_bwd_dkdv_kernel": seg[2], "fa_bwd_dq_convert_kernel": seg[3]},
+            "fwd_tflops": f_fwd / (seg[0] * 1e-3) / 1e12, "dkdv_tflops": f_bwd / (seg[2] * 1e-3) / 1e12,
+            "config": {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d, "causal": w.causal, "seed": w.seed + rank},
+        }
+        del run
+        torch.cuda.empty_cache()
+    w = WORKLOADS[5]
+    dec = _DecodeRun(lib, fa, w, dev, w.seed + rank)
+    steps = args.extra_steps * 10
+    ms = max_over_ranks(dec.timed(steps, 3, barrier), dist, dev) / steps
+    value = world * dec.alg_bytes / (ms * 1e-3) / 1e9
+    out[w.name] = {
+        "metric": "split-KV decode HBM GB/s (bf16 KV cache, 1xB200) and % of HBM peak", "value": value,
+        "unit": "GB/s", "ms_per_step": ms, "steps": steps, "warmup": 3, "frac": value / world / peaks["hbm_gbs"],
+        "tokens_per_s": world * w.B / (ms * 1e-3),
+        "config": {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Tk_max": w.T, "d": w.d, "chunk": w.chunk,
+                   "total_cached_tokens": dec.total_keys, "seed": w.seed + rank},
+    }
+    del dec
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_fa(args, w, rank, world, dist):
-    import ctypes
     import torch
     import io_aware_exact_forward_b200 as fa
-    from workloads import prefill_inputs
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     lib = fa.load_library()
-    inp = prefill_inputs(w, device=dev, seed=w.seed + rank)
-    q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
+    run = _PrefillRun(lib, fa, w, dev, w.seed + rank)
+    q, k, v, do, o, lse, dq, dk, dv, ws = (run.q, run.k, run.v, run.do, run.o, run.lse, run.dq, run.dk, run.dv,
+                                           run.ws)
     B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws_bytes = lib.fa_backward_workspace_bytes(B, Hq, Hkv, T, T, d)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    P = ctypes.c_void_p
-    pq, pk, pv, pdo, po, plse = (P(t.data_ptr()) for t in (q, k, v, do, o, lse))
-    pdq, pdk, pdv, pws = (P(t.data_ptr()) for t in (dq, dk, dv, ws))
-    stream = torch.cuda.current_stream(dev)
-    sp = P(stream.cuda_stream)
-    scale, causal = w.scale, int(w.causal)
-    # with a sliding window the windowed entry points take the window in
-    # place of the causal flag
-    fwd_fn, dkdv_fn, mask_arg = lib.fa_forward, lib.fa_backward_dkdv, causal
-    if w.window:
-        fwd_fn, dkdv_fn, mask_arg = lib.fa_forward_window, lib.fa_backward_dkdv_window, w.window
-
-    def check(st, name):
-        if st != 0:
-            raise RuntimeError(f"{name}: {fa.STATUS.get(st, st)}")
-
-    def step(evs=None):
-        if evs: evs[0].record(stream)
-        check(fwd_fn(pq, pk, pv, po, plse, B, Hq, Hkv, T, T, d, scale, mask_arg, sp), "fa_forward")
-        if evs: evs[1].record(stream)
-        check(lib.fa_backward_preprocess(po, plse, pdo, pws, ws_bytes, B, Hq, Hkv, T, T, d, sp), "preprocess")
-        if evs: evs[2].record(stream)
-        check(dkdv_fn(pq, pk, pv, pdo, pdk, pdv, pws, ws_bytes, B, Hq, Hkv, T, T, d, scale, mask_arg, sp),
-              "dkdv")
-        if evs: evs[3].record(stream)
-        check(lib.fa_backward_dq_finalize(pdq, pws, ws_bytes, B, Hq, Hkv, T, T, d, sp), "dq_finalize")
-        if evs: evs[4].record(stream)
-
-    kernels_per_step = 4
+    scale = w.scale
+    kernels_per_step = run.KERNELS_PER_STEP
 
     def barrier():
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    for _ in range(args.warmup):
-        step()
-    barrier()
-    if lib.fa_check(sp) != 0:
-        raise RuntimeError("device status set during warm-up")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     gpu_index = local
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -520,18 +620,9 @@ def run_fa(args, w, rank, world, dist):
             gpu_index = int(vis.split(",")[local])
         except ValueError:
             pass
-    barrier()
     with ClockSampler(gpu_index) as clocks:
-        t_start.record(stream)
-        for s in range(args.steps):
-            step(evs[s])
-        t_end.record(stream)
-        barrier()
-    status = lib.fa_check(sp)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
-    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
-    seg = [sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps for i in range(4)]
+        elapsed_ms, seg = run.timed(args.steps, args.warmup, barrier)
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
     ms_per_step = elapsed_ms / args.steps
     f_fwd, f_bwd = flops(w)
     value = job_rate(f_fwd + f_bwd, world, args.steps, elapsed_ms) / 1e12
@@ -622,24 +713,33 @@ def run_fa(args, w, rank, world, dist):
         barrier()
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
         e2e = {"value": job_rate(f_fwd + f_bwd, world, args.e2e_steps, e_ms) / 1e12, "unit": "TFLOP/s",
+               "tokens_per_s": world * prefill_tokens(w) * args.e2e_steps / (e_ms * 1e-3),
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "ms_per_step": e_ms / args.e2e_steps,
                "pipelining": "two device slots; copies of neighbouring steps overlap compute on separate streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        inp_cpu = {n: inp[n].cpu() for n in ("q", "k", "v", "do")}
+        inp_cpu = {"q": q.cpu(), "k": k.cpu(), "v": v.cpu(), "do": do.cpu()}
         cpu = cpu_baseline(w, inp_cpu, args.cpu_seconds)
+        cpu["tokens_per_s"] = cpu["value"] * 1e12 / ((f_fwd + f_bwd) / prefill_tokens(w))
+
+    extras = None
+    if args.workload == 2 and not w.window and args.batch is None and not args.no_extra:
+        del run, q, k, v, do, o, lse, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+        extras = extra_workloads(args, lib, fa, dev, rank, world, dist, barrier)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "tokens_per_s": world * prefill_tokens(w) / (ms_per_step * 1e-3),
             "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
                        "window": w.window or None,
                        "step": "fa_forward + fa_backward (preprocess, dkdv, dq_finalize)",
-                       "l2": "inputs larger than L2 (q, k, v, dO: 4 x %d MiB per step)" % (q.numel() * 2 >> 20),
+                       "l2": "inputs larger than L2 (q, k, v, dO: 4 x %d MiB per step)" % (B * T * Hq * d * 2 >> 20),
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "seed": w.seed},
             "pct_of_peak": {"measured": value / world / peaks["bf16_tflops"], "spec_2250": value / world / 2250.0},
@@ -649,72 +749,94 @@ def run_fa(args, w, rank, world, dist):
             "e2e": e2e,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clocks.summary(),
+            "workloads": extras,
         }
         print(json.dumps(line), flush=True)
     return 0
+
+
+class _DecodeRun:
+    """Device buffers and the launch of one split-KV decode step, called
+    through the C ABI."""
+
+    def __init__(self, lib, fa, w, dev, seed):
+        import ctypes
+        import torch
+        from workloads import decode_inputs
+        self.fa, self.lib, self.w, self.dev = fa, lib, w, dev
+        inp = decode_inputs(w, device=dev, seed=seed)
+        self.q, self.kc, self.vc, self.sl = inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"]
+        B, Hq, Hkv, Tk_max, d, chunk = w.B, w.Hq, w.Hkv, w.T, w.d, w.chunk
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        self.wsb = lib.fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk)
+        self.ws = torch.empty(self.wsb, dtype=torch.uint8, device=dev)
+        P = ctypes.c_void_p
+        self.stream = torch.cuda.current_stream(dev)
+        self.sp = P(self.stream.cuda_stream)
+        args_c = (P(self.q.data_ptr()), P(self.kc.data_ptr()), P(self.vc.data_ptr()), P(self.sl.data_ptr()),
+                  P(self.o.data_ptr()), P(self.lse.data_ptr()), P(self.ws.data_ptr()), self.wsb, B, Hq, Hkv,
+                  Tk_max, d, w.scale, chunk)
+        self.fn = lib.fa_decode_splitkv
+        if w.window:
+            self.fn = lib.fa_decode_splitkv_window
+            args_c = args_c + (w.window,)
+        self.args_c = args_c + (self.sp,)
+        # keys the query sees: the whole prefix, or its last `window` keys
+        sl = self.sl
+        self.total_keys = int(sl.clamp(max=w.window).sum().item()) if w.window else int(sl.sum().item())
+        self.alg_bytes = (self.total_keys * Hkv * d * 2 * 2 + self.q.numel() * 2 + self.o.numel() * 2
+                          + self.lse.numel() * 4)
+
+    def step(self):
+        st = self.fn(*self.args_c)
+        if st != 0:
+            raise RuntimeError(f"fa_decode_splitkv: {self.fa.STATUS.get(st, st)}")
+
+    KERNELS_PER_STEP = 3   # split, combine, empty-sequence kernels
+
+    def timed(self, steps, warmup, barrier):
+        """Elapsed ms of `steps` decode steps on this rank after `warmup`; the
+        cache (2 x 4.3 GB) is far larger than L2, so no flush is needed."""
+        import torch
+        for _ in range(warmup):
+            self.step()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for _ in range(steps):
+            self.step()
+        e1.record(self.stream)
+        barrier()
+        if self.lib.fa_check(self.sp) != 0:
+            raise RuntimeError("device status set during the timed region")
+        return e0.elapsed_time(e1)
 
 
 def run_decode(args, w, rank, world, dist):
     """Split-KV decode of the B=64, Hq=32, Hkv=8, d=128 batch: one step is
     fa_decode_splitkv (split kernel + combine kernel); value is algorithmic
     HBM GB/s (K and V of every cached token read once, plus q, o, lse)."""
-    import ctypes
     import torch
     import io_aware_exact_forward_b200 as fa
-    from workloads import decode_inputs
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     lib = fa.load_library()
-    inp = decode_inputs(w, device=dev, seed=w.seed + rank)
-    q, kc, vc, sl = inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"]
+    run = _DecodeRun(lib, fa, w, dev, w.seed + rank)
+    q, kc, vc, sl, o, lse, ws = run.q, run.kc, run.vc, run.sl, run.o, run.lse, run.ws
     B, Hq, Hkv, Tk_max, d, chunk = w.B, w.Hq, w.Hkv, w.T, w.d, w.chunk
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
-    wsb = lib.fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk)
-    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
-    P = ctypes.c_void_p
-    stream = torch.cuda.current_stream(dev)
-    sp = P(stream.cuda_stream)
-    args_c = (P(q.data_ptr()), P(kc.data_ptr()), P(vc.data_ptr()), P(sl.data_ptr()), P(o.data_ptr()),
-              P(lse.data_ptr()), P(ws.data_ptr()), wsb, B, Hq, Hkv, Tk_max, d, w.scale, chunk)
-    dec_fn = lib.fa_decode_splitkv
-    if w.window:
-        dec_fn = lib.fa_decode_splitkv_window
-        args_c = args_c + (w.window,)
-    args_c = args_c + (sp,)
-
-    def step():
-        st = dec_fn(*args_c)
-        if st != 0:
-            raise RuntimeError(f"fa_decode_splitkv: {fa.STATUS.get(st, st)}")
-
-    # keys the query sees: the whole prefix, or its last `window` keys
-    total_keys = int(sl.clamp(max=w.window).sum().item()) if w.window else int(sl.sum().item())
-    alg_bytes = total_keys * Hkv * d * 2 * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
+    total_keys, alg_bytes = run.total_keys, run.alg_bytes
 
     def barrier():
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    for _ in range(args.warmup):
-        step()
-    barrier()
-    # the cache (2 x 4.3 GB) is far larger than L2: no flush needed
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    gpu_index = local
-    with ClockSampler(gpu_index) as clocks:
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        barrier()
-    if lib.fa_check(sp) != 0:
-        raise RuntimeError("device status set during the timed region")
-    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    with ClockSampler(local) as clocks:
+        ms = max_over_ranks(run.timed(args.steps, args.warmup, barrier), dist, dev)
     value = job_rate(alg_bytes, world, args.steps, ms) / 1e9
 
     # End to end through the public binding: per step the query rows and the
@@ -739,13 +861,14 @@ def run_decode(args, w, rank, world, dist):
         barrier()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
+        f0.record(run.stream)
         for _ in range(args.e2e_steps):
             e2e_step()
-        f1.record(stream)
+        f1.record(run.stream)
         barrier()
         e_ms = max_over_ranks(f0.elapsed_time(f1), dist, dev)
         e2e = {"value": job_rate(alg_bytes, world, args.e2e_steps, e_ms) / 1e9, "unit": "GB/s",
+               "tokens_per_s": world * B * args.e2e_steps / (e_ms * 1e-3),
                "h2d_bytes_per_step": hq.numel() * hq.element_size() + hsl.numel() * hsl.element_size(),
                "d2h_bytes_per_step": ho.numel() * ho.element_size() + hlse.numel() * hlse.element_size(),
                "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps,
@@ -757,6 +880,7 @@ def run_decode(args, w, rank, world, dist):
         # the oracle over the first two sequences' caches, copied to the host
         nb, dt, nbytes = oracle_decode(w, q[:2].cpu(), kc[:2].cpu(), vc[:2].cpu(), sl[:2].cpu(), args.cpu_seconds)
         cpu = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+               "tokens_per_s": nb / w.Hkv / dt,
                "sample": f"float64 oracle decode of {nb} (sequence, KV head) groups, cycling over the first two "
                          f"sequences of {w.name} ({dt:.1f} s; same algorithmic bytes as the GPU metric)"}
 
@@ -766,6 +890,7 @@ def run_decode(args, w, rank, world, dist):
             "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
+            "tokens_per_s": world * B * args.steps / (ms * 1e-3),
             "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "Tk_max": Tk_max, "d": d, "chunk": chunk,
                        "total_cached_tokens": total_keys, "window": w.window or None,
                        "l2": "KV cache larger than L2", "seed": w.seed},
@@ -894,6 +1019,7 @@ def run_fp8_forward(args, w, rank, world, dist):
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3", "data": "synthetic",
+            "tokens_per_s": world * prefill_tokens(w) * args.steps / (ms * 1e-3),
             "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
                        "inputs": "E4M3 codes, per-tensor amax/448 factors", "l2": "256 MiB flush between launches",
                        "seed": w.seed},
@@ -978,6 +1104,7 @@ def run_dropout_forward(args, w, rank, world, dist):
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
+            "tokens_per_s": world * prefill_tokens(w) * args.steps / (ms * 1e-3),
             "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
                        "dropout": args.dropout, "l2": "256 MiB flush between launches", "seed": w.seed},
             "plain_forward": {"ms_per_step": ms_plain / args.steps,
@@ -1106,6 +1233,7 @@ def run_decode_cp(args, w, rank, world, dist):
             "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
+            "tokens_per_s": B * args.steps / (ms * 1e-3),
             "config": {"workload": w.name, "context_parallel": True, "B": B, "Hq": Hq, "Hkv": Hkv,
                        "Tk_max": Tk_max, "shard_len": shard_len, "d": d, "chunk": chunk,
                        "total_cached_tokens": total_keys, "l2": "KV cache larger than L2", "seed": w.seed},

@@ -214,7 +214,8 @@ size_t fa_decode_workspace_bytes(int B, int Hq, int Tk_max, int d, int chunk);
  * FlashDecoding).
  *   q [B,Hq,d] bf16; k_cache/v_cache [B,Tk_max,Hkv,d] bf16;
  *   seqlens_k: DEVICE int32 [B], each in [0, Tk_max] (sequence b attends to
- *   its first seqlens_k[b] cached keys, no mask);
+ *   its first seqlens_k[b] cached keys, no mask); a value outside that range
+ *   is read as the nearer end of it (below 0 as 0, above Tk_max as Tk_max);
  *   o [B,Hq,d] bf16 out; lse [B,Hq] fp32 out;
  *   ws/ws_bytes: at least fa_decode_workspace_bytes(); contents on entry do
  *   not matter.  chunk must be a positive multiple of 64.
@@ -239,11 +240,11 @@ int fa_decode_splitkv_window(const void* q, const void* k_cache, const void* v_c
 
 /*
  * fa_decode_splitkv_noalloc -- fa_decode_splitkv for callers that cannot
- * allocate device memory where they call it: code running inside a CUDA
- * graph capture or a plug-in interface that only hands over inputs and
- * outputs, or a latency-critical loop that cannot afford cudaMalloc's
- * implicit device synchronisation.  The pages have no counterpart; this is a
- * deployment convenience around the same kernels.
+ * allocate device memory where they call it: a plug-in interface of a
+ * serving engine that hands the kernel its input and output tensors but no
+ * allocator, or a latency-critical decode loop that cannot afford
+ * cudaMalloc's implicit device synchronisation.  The pages have no
+ * counterpart; this is a deployment convenience around the same kernels.
  *   Arguments as for fa_decode_splitkv, without ws/ws_bytes.  The chunk
  *   partials live in a 32 MiB array inside the library (every GPU that loads
  *   the library holds it until the process exits), so

@@ -694,10 +694,9 @@ extern "C" int fa_selftest_bounded_wait(int limit_us, void* stream) {
 // ---------------------------------------------------------------------------
 // Split-KV decode without caller-provided workspace.
 //
-// For callers that cannot allocate device memory at the call site -- code
-// that runs while a CUDA graph is being captured through an API that
-// forbids allocation, plug-in interfaces that hand over only the input and
-// output tensors, or latency-critical loops where cudaMalloc's implicit
+// For callers that cannot allocate device memory at the call site --
+// plug-in interfaces that hand over only the input and output tensors and
+// no allocator, or latency-critical loops where cudaMalloc's implicit
 // device synchronisation is not acceptable.  The chunk partials live in one
 // file-scope device array that every GPU loading this library keeps until
 // the process exits.
@@ -733,7 +732,11 @@ extern "C" int fa_decode_splitkv_noalloc(const void* q, const void* k_cache, con
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   // The partials of this call must fit in the built-in scratch array.
   if (fa_decode_workspace_bytes(B, Hq, Tk_max, d, chunk) > kDecodeScratchBytes) return FA_ERR_WORKSPACE;
-  if (B == 0) return FA_OK;
+  // No rows: the workspace entry point checks the remaining arguments the
+  // same way and returns before it touches the (empty) workspace.
+  if (B == 0)
+    return fa_decode_splitkv(q, k_cache, v_cache, seqlens_k, o, lse, nullptr, 0, B, Hq, Hkv, Tk_max, d, scale, chunk,
+                             stream);
   void* scratch = nullptr;
   const int st = decode_scratch_ptr(&scratch);
   if (st) return st;

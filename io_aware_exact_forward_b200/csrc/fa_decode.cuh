@@ -99,6 +99,12 @@ __device__ __forceinline__ uint32_t swz_off(int key, int ch) {
   return (uint32_t)((ch >> 3) * 64 * 128 + key * 128 + (((ch & 7) ^ (key & 7)) << 4));
 }
 
+// A sequence length as every decode kernel reads it: clamped to
+// [0, Tk_max], so that a length outside the cache's extent can neither send
+// the split kernel past its chunk count nor the merge past the partials the
+// split kernel wrote.
+__device__ __forceinline__ int clamp_seqlen(const DecodeParams& p, int n) { return min(max(n, 0), p.Tk_max); }
+
 // Item k covers chunk k % nchunk of (sequence, KV head) k / nchunk.
 template <int D, int G>
 __global__ void __launch_bounds__(DecCfg<D, G>::THREADS)
@@ -122,7 +128,7 @@ fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
   const int lane = threadIdx.x & 31;
   WaitCtl wc{abort_flag, p.wait_limit_ns};
 
-  for (int i = threadIdx.x; i < min(p.B, C::SEQ_CACHE); i += blockDim.x) seq_s[i] = p.seqlens[i];
+  for (int i = threadIdx.x; i < min(p.B, C::SEQ_CACHE); i += blockDim.x) seq_s[i] = clamp_seqlen(p, p.seqlens[i]);
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     *stop_flag = 0;
@@ -137,7 +143,7 @@ fa_decode_split_kernel(const __grid_constant__ DecodeParams p) {
     fence_barrier_init();
   }
   __syncthreads();
-  auto seqlen_of = [&](int b) { return b < C::SEQ_CACHE ? seq_s[b] : p.seqlens[b]; };
+  auto seqlen_of = [&](int b) { return b < C::SEQ_CACHE ? seq_s[b] : clamp_seqlen(p, p.seqlens[b]); };
 
   if (warp == C::NWARP) {
     // ---------------------------------------------------------- producer
@@ -369,7 +375,7 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const __grid_con
   const int lane = threadIdx.x & 31;
   if (gw >= p.B * p.Hq) return;
   const int b = gw / p.Hq;
-  const int seqlen = p.seqlens[b];
+  const int seqlen = clamp_seqlen(p, p.seqlens[b]);
   const int nch = (seqlen + p.chunk - 1) / p.chunk;
   if (nch == 0) return;  // written by fa_decode_empty_kernel
   // with a window the chunks before the first visible key were skipped
@@ -414,7 +420,7 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const __grid_con
   store_row<D>(p, gw, lane, acc);
 }
 
-// Sequences with no cached key (seqlen 0) get O = 0 and LSE = -inf; every
+// Sequences with no cached key (seqlen <= 0) get O = 0 and LSE = -inf; every
 // other (sequence, head) is written by the merge kernel.
 template <int D>
 __global__ void __launch_bounds__(256) fa_decode_empty_kernel(const __grid_constant__ DecodeParams p) {
@@ -422,7 +428,7 @@ __global__ void __launch_bounds__(256) fa_decode_empty_kernel(const __grid_const
   const int lane = threadIdx.x & 31;
   if (gw >= p.B * p.Hq) return;
   const int b = gw / p.Hq;
-  if (p.seqlens[b] > 0) return;
+  if (clamp_seqlen(p, p.seqlens[b]) > 0) return;
   float zero[D / 32];
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) zero[e] = 0.f;

@@ -3,12 +3,18 @@
 Tolerances (the targets): max|dO| <= 1e-2, mean|dO| <= 1e-3, |dLSE| <= 1e-3,
 relative L2 error of dQ, dK, dV <= 2e-2.
 
-O is returned in bf16, whose spacing is 2^-6 = 0.0156 for |O| in [2, 4) and
-2^-5 in [4, 8): there the absolute 1e-2 bound is finer than one output ulp,
-so no bf16-output kernel can meet it.  The max bound is therefore applied to
-|dO| / max(1, |O_ref|); for |O_ref| <= 1 (almost every element of the
-N(0,1) workloads) this is the absolute bound itself.  The mean bound stays
-absolute."""
+O is returned in bf16.  Where |O_ref| >= 2 one bf16 spacing (2^-6 = 0.0156 on
+[2, 4), 2^-5 on [4, 8)) is already wider than 1e-2, so rounding the exact
+value to the nearest bf16 and one more rounding step of the fp32 arithmetic
+before it can move an element by more than 1e-2 with nothing wrong.  The max
+bound is therefore applied per element as
+
+    |dO| <= max(1e-2, ulp_bf16(|O_ref|)),
+
+which is the stated absolute 1e-2 wherever |O_ref| < 2 (on [1, 2) one ulp is
+2^-7 < 1e-2) and one output ulp above that.  The mean bound stays absolute.
+Every failure message reports the absolute max, the number of elements above
+1e-2 and the worst element's reference value."""
 
 import numpy as np
 
@@ -18,18 +24,37 @@ LSE_MAX_ABS = 1e-3
 GRAD_REL_L2 = 2e-2
 
 
+def ulp_bf16(x):
+    """Spacing of bf16 numbers at |x|: 2^(e - 7) for |x| in [2^e, 2^(e+1))
+    (8 significant bits); 2^-133 below the normal range."""
+    a = np.abs(np.asarray(x, np.float64))
+    _, e = np.frexp(a)                     # a = m 2^e with m in [0.5, 1)
+    return np.where(a >= 2.0 ** -126, np.ldexp(1.0, e - 8), 2.0 ** -133)
+
+
+def o_bound(o_ref):
+    """Per-element bound on |O_gpu - O_ref|: max(1e-2, one bf16 ulp of O_ref)."""
+    return np.maximum(O_MAX_ABS, ulp_bf16(o_ref))
+
+
 def o_errors(o_gpu, o_ref):
-    """(max of |diff|/max(1,|ref|), mean |diff|, max |diff|)."""
+    """(max |diff|, mean |diff|, number of elements with |diff| > 1e-2,
+    number above the per-element bound, worst excess over the bound, |O_ref|
+    at the largest |diff|)."""
     ref = np.asarray(o_ref, np.float64)
     d = np.abs(np.asarray(o_gpu, np.float64) - ref)
     if not d.size:
-        return 0.0, 0.0, 0.0
-    return float((d / np.maximum(1.0, np.abs(ref))).max()), float(d.mean()), float(d.max())
+        return 0.0, 0.0, 0, 0, 0.0, 0.0
+    excess = d - o_bound(ref)
+    i = int(np.argmax(d))
+    return (float(d.max()), float(d.mean()), int((d > O_MAX_ABS).sum()), int((excess > 0).sum()),
+            float(excess.max()), float(np.abs(ref.flat[i])))
 
 
 def assert_o_close(o_gpu, o_ref, what="O"):
-    mx, mean, mx_abs = o_errors(o_gpu, o_ref)
-    assert mx <= O_MAX_ABS, f"{what}: max|diff|/max(1,|O|) {mx:.3e} > {O_MAX_ABS} (abs {mx_abs:.3e})"
+    mx, mean, n_over, n_bad, worst, at = o_errors(o_gpu, o_ref)
+    assert n_bad == 0, (f"{what}: {n_bad} elements beyond max(1e-2, ulp_bf16(|O_ref|)); worst excess {worst:.3e}; "
+                        f"max|diff| {mx:.3e} at |O_ref| = {at:.4g}; {n_over} elements above 1e-2")
     assert mean <= O_MEAN_ABS, f"{what}: mean|diff| {mean:.3e} > {O_MEAN_ABS}"
     return mx, mean
 

@@ -65,3 +65,23 @@ def test_decode_splitkv_b64_hq32_hkv8_d128_sampled():
                                      to_f64(inp["v_cache"][b, :n, g]), w.scale, False)
         assert_o_close(to_f64(o[b, h])[None], Ob, what=f"O[{b},{h}]")
         assert_lse_close(lse[b, h].cpu().numpy()[None], Lb, what=f"LSE[{b},{h}]")
+
+
+def test_decode_lengths_outside_the_cache_are_clamped():
+    """A seqlens entry above Tk_max reads as Tk_max and one below 0 as 0:
+    the result equals the run with the clamped lengths (bit for bit, the same
+    kernels on the same data), and no kernel reads past the partials its
+    own call wrote."""
+    w = WORKLOADS[5].with_(Hq=8, Hkv=2, d=128)
+    inp = decode_inputs(w, seed=31, B=3, Tk_max=700, seqlens=[700, 300, 0])
+    dev = {k: v.cuda() for k, v in inp.items()}
+    bad = torch.tensor([700 + 5000, 300, -17], dtype=torch.int32, device="cuda")
+    o_bad, lse_bad = fa.decode_splitkv(dev["q"], dev["k_cache"], dev["v_cache"], bad, scale=w.scale, chunk=256)
+    o_ok, lse_ok = fa.decode_splitkv(dev["q"], dev["k_cache"], dev["v_cache"], dev["seqlens"], scale=w.scale,
+                                     chunk=256)
+    assert fa.check() == 0
+    assert torch.equal(o_bad, o_ok)
+    assert torch.equal(lse_bad, lse_ok)
+    O, LSE = _oracle(inp, w)
+    assert_o_close(to_f64(o_bad), O)
+    assert_lse_close(lse_bad.cpu().numpy(), LSE)

@@ -59,7 +59,8 @@ def parse_args():
     ap.add_argument("--fp8", action="store_true",
                     help="prefill, d = 128 only: the E4M3 forward (fa_forward_fp8) alone")
     ap.add_argument("--dropout", type=float, default=None,
-                    help="prefill: the forward with fused dropout of this rate alone (fa_forward_dropout)")
+                    help="prefill: forward + backward with fused dropout of this rate (fa_forward_dropout, "
+                         "fa_backward_dkdv_dropout)")
     ap.add_argument("--cp", action="store_true",
                     help="decode only: context-parallel, every sequence's cache cut into one share per GPU")
     ap.add_argument("--batch", type=int, default=None,
@@ -362,21 +363,21 @@ def run_reference_fp8(args, w):
 
 
 def run_reference_dropout(args, w):
-    """The oracle's forward with dropout on P on the host cores: each step
-    one (batch, head) of the workload (heads cycling)."""
-    import oracle
+    """The oracle's forward + backward with dropout on P on the host cores:
+    each step one (batch, head) of the workload (heads cycling)."""
     from oracle import dropout as dr
     from workloads import prefill_inputs, to_f64
     inp = prefill_inputs(w.with_(B=1), device="cpu")
     G = w.Hq // w.Hkv
-    f_fwd, _ = flops(w)
-    per_head = f_fwd / (w.B * w.Hq)
+    f_fwd, f_bwd = flops(w)
+    per_head = (f_fwd + f_bwd) / (w.B * w.Hq)
 
     def one(s):
         h = s % w.Hq
+        qh, kh, vh, dh = (to_f64(inp[n][0, :, h if n in ("q", "do") else h // G]) for n in ("q", "k", "v", "do"))
         t0 = time.perf_counter()
-        dr.head_forward_dropout(to_f64(inp["q"][0, :, h]), to_f64(inp["k"][0, :, h // G]),
-                                to_f64(inp["v"][0, :, h // G]), w.scale, w.causal, args.dropout, 0x5EED0000, s, h)
+        dr.head_forward_dropout(qh, kh, vh, w.scale, w.causal, args.dropout, 0x5EED0000, 0, h)
+        dr.head_backward_dropout(qh, kh, vh, dh, w.scale, w.causal, args.dropout, 0x5EED0000, 0, h)
         return time.perf_counter() - t0
 
     for s in range(args.warmup):
@@ -385,13 +386,14 @@ def run_reference_dropout(args, w):
     value = per_head * args.steps / tot / 1e12
     line = {
         "impl": "reference",
-        "metric": "attention forward TFLOPS with fused dropout (bf16, 1xB200) and % of dense tensor peak",
+        "metric": "attention fwd+bwd TFLOPS with fused dropout (bf16, 1xB200) and % of dense tensor peak",
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "tokens_per_s": tokens_at_rate(value, f_fwd, prefill_tokens(w)),
+        "tokens_per_s": tokens_at_rate(value, f_fwd + f_bwd, prefill_tokens(w)),
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d, "causal": w.causal,
-                   "dropout": args.dropout, "step": "one (batch, head) of the workload, forward with dropout"},
+                   "dropout": args.dropout,
+                   "step": "one (batch, head) of the workload, forward and backward with dropout"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": f"one (batch, head) of {w.name} per step, float64 numpy"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -464,7 +466,7 @@ class _PrefillRun:
     """Device buffers and the four launches of one fwd+bwd step of a prefill
     workload, called through the C ABI."""
 
-    def __init__(self, lib, fa, w, dev, seed):
+    def __init__(self, lib, fa, w, dev, seed, dropout=None):
         import ctypes
         import torch
         from workloads import prefill_inputs
@@ -484,10 +486,15 @@ class _PrefillRun:
         self.stream = torch.cuda.current_stream(dev)
         self.sp = P(self.stream.cuda_stream)
         # with a sliding window the windowed entry points take the window in
-        # place of the causal flag
+        # place of the causal flag; with dropout the dropout entry points take
+        # (rate, seed, offset) after it
         self.fwd_fn, self.dkdv_fn, self.mask_arg = lib.fa_forward, lib.fa_backward_dkdv, int(w.causal)
+        self.extra = ()
         if w.window:
             self.fwd_fn, self.dkdv_fn, self.mask_arg = lib.fa_forward_window, lib.fa_backward_dkdv_window, w.window
+        if dropout is not None:
+            self.fwd_fn, self.dkdv_fn = lib.fa_forward_dropout, lib.fa_backward_dkdv_dropout
+            self.extra = (float(dropout), 0x5EED0000 + seed, 0)
 
     def _check(self, st, name):
         if st != 0:
@@ -498,13 +505,13 @@ class _PrefillRun:
         B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
         if evs: evs[0].record(s)
         self._check(self.fwd_fn(self.pq, self.pk, self.pv, self.po, self.plse, B, Hq, Hkv, T, T, d, w.scale,
-                                self.mask_arg, self.sp), "fa_forward")
+                                self.mask_arg, *self.extra, self.sp), "fa_forward")
         if evs: evs[1].record(s)
         self._check(lib.fa_backward_preprocess(self.po, self.plse, self.pdo, self.pws, self.ws_bytes, B, Hq, Hkv, T,
                                                T, d, self.sp), "preprocess")
         if evs: evs[2].record(s)
         self._check(self.dkdv_fn(self.pq, self.pk, self.pv, self.pdo, self.pdk, self.pdv, self.pws, self.ws_bytes,
-                                 B, Hq, Hkv, T, T, d, w.scale, self.mask_arg, self.sp), "dkdv")
+                                 B, Hq, Hkv, T, T, d, w.scale, self.mask_arg, *self.extra, self.sp), "dkdv")
         if evs: evs[3].record(s)
         self._check(lib.fa_backward_dq_finalize(self.pdq, self.pws, self.ws_bytes, B, Hq, Hkv, T, T, d, self.sp),
                     "dq_finalize")
@@ -1036,85 +1043,66 @@ def run_fp8_forward(args, w, rank, world, dist):
     return 0
 
 
-def run_dropout_forward(args, w, rank, world, dist):
-    """The forward with fused dropout on P (rate args.dropout) on a prefill
-    workload: one step is one fa_forward_dropout launch (inputs resident, L2
-    flushed between launches).  value is algorithmic TFLOP/s (4 B Hq d
-    pairs, the dropout's mask work not counted); the plain forward is timed
-    the same way in the same run for the overhead."""
-    import ctypes
+def run_dropout(args, w, rank, world, dist):
+    """Forward + backward with fused dropout on P (rate args.dropout) on a
+    prefill workload: one step is fa_forward_dropout + the three backward
+    steps with fa_backward_dkdv_dropout (inputs resident, larger than L2).
+    value is algorithmic TFLOP/s (14 B Hq d pairs; the mask's work is not
+    counted).  The plain fwd+bwd step is timed the same way in the same run
+    for the overhead."""
     import torch
     import io_aware_exact_forward_b200 as fa
-    from workloads import prefill_inputs
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     lib = fa.load_library()
-    inp = prefill_inputs(w, device=dev, seed=w.seed + rank)
-    q, k, v = inp["q"], inp["k"], inp["v"]
-    B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
-    P = ctypes.c_void_p
-    stream = torch.cuda.current_stream(dev)
-    sp = P(stream.cuda_stream)
-    base = (P(q.data_ptr()), P(k.data_ptr()), P(v.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
-            B, Hq, Hkv, T, T, d, w.scale, int(w.causal))
-    seed = 0x5EED0000 + rank
-
-    def step(s_, drop=True):
-        st = (lib.fa_forward_dropout(*base, float(args.dropout), seed, s_, sp) if drop
-              else lib.fa_forward(*base, sp))
-        if st != 0:
-            raise RuntimeError(f"forward: {fa.STATUS.get(st, st)}")
 
     def barrier():
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-
-    def timed(drop):
-        for s_ in range(args.warmup):
-            step(s_, drop)
-        barrier()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        for s_ in range(args.steps):
-            flush.fill_(s_ & 0xFF)
-            evs[s_][0].record(stream)
-            step(s_, drop)       # a new offset every step: a new mask
-            evs[s_][1].record(stream)
-        barrier()
-        return max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), dist, dev)
-
+    run = _PrefillRun(lib, fa, w, dev, w.seed + rank, dropout=args.dropout)
     with ClockSampler(local) as clocks:
-        ms = timed(True)
-    ms_plain = timed(False)
-    if lib.fa_check(sp) != 0:
-        raise RuntimeError("device status set during the timed region")
-    f_fwd, _ = flops(w)
-    value = job_rate(f_fwd, world, args.steps, ms) / 1e12
+        elapsed, seg = run.timed(args.steps, args.warmup, barrier)
+    del run
+    plain = _PrefillRun(lib, fa, w, dev, w.seed + rank)
+    elapsed_plain, seg_plain = plain.timed(args.steps, args.warmup, barrier)
+    del plain
+    elapsed = max_over_ranks(elapsed, dist, dev)
+    elapsed_plain = max_over_ranks(elapsed_plain, dist, dev)
+    f_fwd, f_bwd = flops(w)
+    value = job_rate(f_fwd + f_bwd, world, args.steps, elapsed) / 1e12
+    ms = elapsed / args.steps
     peaks = load_peaks()
+    names = ["fa_fwd_kernel<d, false, true>", "fa_bwd_preprocess_kernel", "fa_bwd_dkdv_kernel<d, false, true>",
+             "fa_bwd_dq_convert_kernel"]
+    dom = max(range(4), key=lambda i: seg[i])
+    alg = f_fwd if dom == 0 else (f_bwd if dom == 2 else None)
     if rank == 0:
         line = {
-            "metric": "attention forward TFLOPS with fused dropout (bf16, 1xB200) and % of dense tensor peak",
+            "metric": "attention fwd+bwd TFLOPS with fused dropout (bf16, 1xB200) and % of dense tensor peak",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "tokens_per_s": world * prefill_tokens(w) * args.steps / (ms * 1e-3),
-            "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
-                       "dropout": args.dropout, "l2": "256 MiB flush between launches", "seed": w.seed},
-            "plain_forward": {"ms_per_step": ms_plain / args.steps,
-                              "tflops": job_rate(f_fwd, world, args.steps, ms_plain) / 1e12},
-            "roofline": {"kernel": "fa_fwd_kernel<d, false, true>", "bound": "tensor", "achieved": value / world,
+            "tokens_per_s": world * prefill_tokens(w) / (ms * 1e-3),
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d,
+                       "causal": w.causal, "dropout": args.dropout,
+                       "step": "fa_forward_dropout + preprocess + fa_backward_dkdv_dropout + dq_finalize",
+                       "l2": "inputs larger than L2", "seed": w.seed},
+            "per_kernel_ms": {names[i]: seg[i] for i in range(4)},
+            "fwd_tflops": f_fwd / (seg[0] * 1e-3) / 1e12, "dkdv_tflops": f_bwd / (seg[2] * 1e-3) / 1e12,
+            "plain": {"ms_per_step": elapsed_plain / args.steps,
+                      "tflops": job_rate(f_fwd + f_bwd, world, args.steps, elapsed_plain) / 1e12,
+                      "per_kernel_ms": seg_plain},
+            "roofline": {"kernel": names[dom], "bound": "tensor" if alg else "hbm",
+                         "achieved": alg / (seg[dom] * 1e-3) / 1e12 if alg else None,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": value / world / peaks["bf16_tflops"],
+                         "frac": alg / (seg[dom] * 1e-3) / 1e12 / peaks["bf16_tflops"] if alg else None,
                          "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": None,
-                         "algorithmic_per_launch": f_fwd},
-            "gpu_launches": args.steps,
+                         "algorithmic_per_launch": alg},
+            "gpu_launches": _PrefillRun.KERNELS_PER_STEP * args.steps,
             "clocks": clocks.summary(),
             "cpu_baseline": None,
             "e2e": None,
@@ -1290,7 +1278,7 @@ def main():
         if args.fp8:
             return run_fp8_forward(args, w, rank, world, dist)
         if args.dropout is not None:
-            return run_dropout_forward(args, w, rank, world, dist)
+            return run_dropout(args, w, rank, world, dist)
         if w.decode and args.cp:
             return run_decode_cp(args, w, rank, world, dist)
         if w.decode:

@@ -202,6 +202,33 @@ int fa_backward_dq_finalize(void* dq, void* ws, size_t ws_bytes, int B, int Hq, 
                             int d, void* stream);
 
 /*
+ * fa_backward_dropout -- gradients of L = sum(dO * O) for fa_forward_dropout
+ * with the same p_drop, seed and offset ("Efficient attention: memory-bound",
+ * "Real code moves even more": dropout on P before the final product; the
+ * products are those of fa_backward with the keep mask Z in them):
+ *   dV = s (P*Z)^T dO,  dP = s (dO V^T) * Z,  dS = P * (dP - D),
+ *   dQ = scale dS K,    dK = scale dS^T Q,    s = 256 / t,
+ * with D_i = sum_c dO_ic O_ic of the dropout forward's O (equal to
+ * sum_j P_ij dP_ij) and P recomputed from its (undropped) LSE.  Z is not
+ * stored: the kernel regenerates the forward's Philox-4x32-10 mask block by
+ * block, so o and lse must come from fa_forward_dropout with the same
+ * (p_drop, seed, offset).  p_drop = 0 gives fa_backward.  Arguments,
+ * workspace, layouts and errors as fa_backward; p_drop outside [0, 1) is
+ * FA_ERR_INVALID_ARG.  bf16 only; no window.
+ *
+ * fa_backward_dkdv_dropout -- its dK/dV step alone (after
+ * fa_backward_preprocess, before fa_backward_dq_finalize).
+ */
+int fa_backward_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B, int Hq,
+                        int Hkv, int Tq, int Tk, int d, float scale, int causal, float p_drop,
+                        unsigned long long seed, unsigned int offset, void* stream);
+int fa_backward_dkdv_dropout(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                             void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+                             float scale, int causal, float p_drop, unsigned long long seed, unsigned int offset,
+                             void* stream);
+
+/*
  * Bytes of device workspace fa_decode_splitkv needs: fp32 partial outputs
  * [B,Hq,nchunk,d] and partial LSEs [B,Hq,nchunk], nchunk = ceil(Tk_max/chunk).
  */

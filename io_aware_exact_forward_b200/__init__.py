@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     SIGNATURES,
     STATUS,
     backward,
+    backward_dropout,
     backward_workspace_bytes,
     check,
     decode_merge,

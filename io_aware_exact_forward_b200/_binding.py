@@ -39,6 +39,11 @@ SIGNATURES = {
     "fa_backward_workspace_bytes": (_c_size, [_c_int] * 6),
     "fa_backward": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_window": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_backward_dropout": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _c_float,
+                                                                             ctypes.c_ulonglong, ctypes.c_uint, _vp]),
+    "fa_backward_dkdv_dropout": (_c_int, [_vp] * 7 + [_c_size] + [_c_int] * 6 + [_c_float, _c_int, _c_float,
+                                                                                ctypes.c_ulonglong, ctypes.c_uint,
+                                                                                _vp]),
     "fa_backward_preprocess": (_c_int, [_vp] * 4 + [_c_size] + [_c_int] * 6 + [_vp]),
     "fa_backward_dkdv": (_c_int, [_vp] * 7 + [_c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_dkdv_window": (_c_int, [_vp] * 7 + [_c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
@@ -219,6 +224,34 @@ def backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None, dq=N
     else:
         st = lib.fa_backward_window(*args, int(window), _stream_ptr(dev))
         _raise("fa_backward_window", st)
+    return dq, dk, dv
+
+
+def backward_dropout(q, k, v, o, lse, do, p_drop, seed, offset=0, scale=None, causal=False, workspace=None,
+                     dq=None, dk=None, dv=None):
+    """dQ, dK, dV for forward_dropout with the same (p_drop, seed, offset):
+    the kernel regenerates the forward's keep mask.  o and lse are the
+    dropout forward's outputs."""
+    lib = load_library()
+    B, Tq, Hq, d = q.shape
+    Tk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_dev(n, t, torch.bfloat16, dev)
+    _check_dev("lse", lse, torch.float32, dev)
+    if scale is None:
+        scale = d ** -0.5
+    need = backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib.fa_backward_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tq, Tk, d, float(scale),
+                                 int(bool(causal)), float(p_drop), int(seed) & (2 ** 64 - 1),
+                                 int(offset) & 0xFFFFFFFF, _stream_ptr(dev))
+    _raise("fa_backward_dropout", st)
     return dq, dk, dv
 
 

@@ -205,6 +205,14 @@ int fa_version(void) { return 100; }
 
 }  // extern "C"
 
+// Dropout keep threshold t = round(256 (1 - p)) clamped to [1, 256]; 256
+// means no dropout.  Returns 0 for a rate outside [0, 1).
+static uint32_t keep_threshold(float p_drop) {
+  if (!(p_drop >= 0.f && p_drop < 1.f)) return 0;
+  long t = lrintf(256.f * (1.f - p_drop));
+  return (uint32_t)(t < 1 ? 1 : (t > 256 ? 256 : t));
+}
+
 // window > 0: sliding window of that many keys (the caller passes causal = 1).
 // f8: q, k, v are E4M3; `qk_factor` multiplies the scores' scale and
 // `o_scale` the output (the dequantising factors).  drop_t in 1..255: dropout
@@ -282,9 +290,8 @@ int fa_forward_window(const void* q, const void* k, const void* v, void* o, floa
 int fa_forward_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                        int Hkv, int Tq, int Tk, int d, float scale, int causal, float p_drop,
                        unsigned long long seed, unsigned int offset, void* stream) {
-  if (!(p_drop >= 0.f && p_drop < 1.f)) return FA_ERR_INVALID_ARG;
-  long t = lrintf(256.f * (1.f - p_drop));
-  t = t < 1 ? 1 : (t > 256 ? 256 : t);
+  const uint32_t t = keep_threshold(p_drop);
+  if (!t) return FA_ERR_INVALID_ARG;
   return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0, stream, false, 1.f,
                       256.f / (float)t, (uint32_t)t, (uint32_t)(seed & 0xFFFFFFFFull), (uint32_t)(seed >> 32),
                       offset);
@@ -362,9 +369,13 @@ int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void
 
 }  // extern "C"
 
+// drop_t in 1..255: dropout on P with that keep threshold and Philox key
+// (seed_lo, seed_hi), counter word drop_offset (the forward's mask).
 static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* ws,
                      size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal,
-                     int window, void* stream) {
+                     int window, void* stream, uint32_t drop_t = 256, uint32_t seed_lo = 0, uint32_t seed_hi = 0,
+                     uint32_t drop_offset = 0) {
+  const bool drop = drop_t < 256;
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
   if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
@@ -396,6 +407,11 @@ static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_kv_tiles = (Tk + 127) / 128;
   p.n_items = p.n_kv_tiles * B * Hkv;
+  p.drop_t = drop_t;
+  p.seed_lo = seed_lo;
+  p.seed_hi = seed_hi;
+  p.drop_offset = drop_offset;
+  p.drop_scale = 256.f / (float)drop_t;
   p.wait_limit_ns = kWaitLimitNs;
   // Non-causal d = 64: one persistent CTA per SM, whose next item's K/V
   // load overlaps the current item (two K/V buffers); items are all the
@@ -407,7 +423,13 @@ static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO
   const bool persistent = d == 64 && !causal;
   dim3 grid(persistent ? std::min(p.n_items, nsm) : p.n_items);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) {
+  if (drop && window > 0) return FA_ERR_UNSUPPORTED;
+  if (drop) {
+    if (d == 64)
+      fa_bwd_dkdv_kernel<64, false, true><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+    else
+      fa_bwd_dkdv_kernel<128, false, true><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+  } else if (d == 64) {
     if (window > 0)
       fa_bwd_dkdv_kernel<64, true><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
     else
@@ -436,6 +458,16 @@ int fa_backward_dkdv_window(const void* q, const void* k, const void* v, const v
   return dkdv_impl(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, 1, window, stream);
 }
 
+int fa_backward_dkdv_dropout(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                             void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+                             float scale, int causal, float p_drop, unsigned long long seed, unsigned int offset,
+                             void* stream) {
+  const uint32_t t = keep_threshold(p_drop);
+  if (!t) return FA_ERR_INVALID_ARG;
+  return dkdv_impl(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0, stream, t,
+                   (uint32_t)(seed & 0xFFFFFFFFull), (uint32_t)(seed >> 32), offset);
+}
+
 int fa_backward_dq_finalize(void* dq, void* ws, size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk,
                             int d, void* stream) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, 1.f, 0);
@@ -455,7 +487,9 @@ int fa_backward_dq_finalize(void* dq, void* ws, size_t ws_bytes, int B, int Hq, 
 
 static int backward_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
                          const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B, int Hq,
-                         int Hkv, int Tq, int Tk, int d, float scale, int causal, int window, void* stream) {
+                         int Hkv, int Tq, int Tk, int d, float scale, int causal, int window, void* stream,
+                         uint32_t drop_t = 256, uint32_t seed_lo = 0, uint32_t seed_hi = 0,
+                         uint32_t drop_offset = 0) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
   if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
@@ -464,7 +498,8 @@ static int backward_impl(const void* q, const void* k, const void* v, const void
   if (Tk > 0 && (st = check_ptrs({k, v, dk, dv}))) return st;
   if ((st = check_ws(ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d))) return st;
   if ((st = fa_backward_preprocess(o, lse, dO, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream))) return st;
-  if ((st = dkdv_impl(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, window, stream)))
+  if ((st = dkdv_impl(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, window, stream,
+                      drop_t, seed_lo, seed_hi, drop_offset)))
     return st;
   return fa_backward_dq_finalize(dq, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream);
 }
@@ -476,6 +511,16 @@ int fa_backward(const void* q, const void* k, const void* v, const void* o, cons
                 int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal, void* stream) {
   return backward_impl(q, k, v, o, lse, dO, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0,
                        stream);
+}
+
+int fa_backward_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B, int Hq,
+                        int Hkv, int Tq, int Tk, int d, float scale, int causal, float p_drop,
+                        unsigned long long seed, unsigned int offset, void* stream) {
+  const uint32_t t = keep_threshold(p_drop);
+  if (!t) return FA_ERR_INVALID_ARG;
+  return backward_impl(q, k, v, o, lse, dO, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, 0,
+                       stream, t, (uint32_t)(seed & 0xFFFFFFFFull), (uint32_t)(seed >> 32), offset);
 }
 
 int fa_backward_window(const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -139,6 +139,11 @@ struct BwdParams {
   float scale, scale_log2;
   int n_kv_tiles;
   int n_items;         // n_kv_tiles * B * Hkv
+  // dropout on P (the DROP instantiation): keep iff the Philox byte < drop_t
+  // (1..255), kept values scaled by drop_scale = 256 / drop_t; Philox key
+  // (seed_lo, seed_hi) and counter word 3 drop_offset, as in the forward
+  uint32_t drop_t, seed_lo, seed_hi, drop_offset;
+  float drop_scale;
   unsigned long long wait_limit_ns;
 };
 
@@ -245,9 +250,50 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
   return it;
 }
 
+// Keep bits of key row `key` for the 64 queries q0 .. q0 + 63 (q0 a multiple
+// of 16) under the forward's dropout mask: bit i of mask[i >> 5] is query
+// q0 + i.  The block of queries 4a..4a+3 and keys 4c..4c+3 is Philox at
+// counter (a, c, bh, offset); word w is query 4a + w, byte j key 4c + j.
+// The four lanes of a quad hold keys 4c..4c+3 (key & 3 == lane & 3): lane q
+// computes the blocks of query groups 4m + q, transposes each block's 4 x 4
+// bytes so that word r holds key 4c + r's bytes, and passes word r to
+// quad-mate r.
+__device__ __forceinline__ void dropout_keep_keyrow_64(uint32_t (&mask)[2], int key, int q0, uint32_t bh,
+                                                       uint32_t offset, uint32_t k0, uint32_t k1, uint32_t t) {
+  const int lane = threadIdx.x & 31;
+  const int q = lane & 3;
+  const uint32_t tt = t * 0x01010101u;
+  mask[0] = mask[1] = 0u;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const uint4 wv = philox4x32_10(make_uint4((uint32_t)(q0 >> 2) + 4 * m + q, (uint32_t)key >> 2, bh, offset), k0, k1);
+    // 4 x 4 byte transpose: x[r] = byte r of words 0..3
+    const uint32_t lo01 = __byte_perm(wv.x, wv.y, 0x5140), hi01 = __byte_perm(wv.x, wv.y, 0x7362);
+    const uint32_t lo23 = __byte_perm(wv.z, wv.w, 0x5140), hi23 = __byte_perm(wv.z, wv.w, 0x7362);
+    const uint32_t x[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
+                           __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int src = (q + s) & 3;       // lane whose block (query group 4m + src) arrives now
+      const int want = (q - s) & 3;      // the key (quad-mate) this lane sends to
+      const uint32_t send = want == 0 ? x[0] : want == 1 ? x[1] : want == 2 ? x[2] : x[3];
+      const uint32_t got = s == 0 ? send : __shfl_sync(0xffffffffu, send, (lane & ~3) | src);
+      const uint32_t lt = __vcmpltu4(got, tt);   // 0xFF in each byte below t
+      const uint32_t bits = ((lt >> 7) & 1u) | ((lt >> 14) & 2u) | ((lt >> 21) & 4u) | ((lt >> 28) & 8u);
+      // queries 4 (4m + src) .. + 3 of the 64: word m / 2, bits 16 (m & 1) + 4 src
+      mask[m >> 1] |= bits << (16 * (m & 1) + 4 * src);
+    }
+  }
+}
+
 // WIN: sliding-window masking compiled in (a separate instantiation, so
-// that the plain path keeps its registers).
-template <int D, bool WIN>
+// that the plain path keeps its registers).  DROP: dropout on P, with the
+// keep mask of the forward regenerated per key row; the P^T warps write the
+// dropped P^T (the dV operand) and the undropped P^T side by side, 8 columns
+// each per 16-query chunk, and the dS warps read the keep bits off the
+// dropped copy's zeros:
+//   dV += (P*Z)^T dO * s,   dS = P * (Z * s * dP - D),   s = 256 / t.
+template <int D, bool WIN, bool DROP = false>
 __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -447,8 +493,11 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             issue_s(gi + 1, kvb_next);
           }
           // P^T of query half h sits in columns [64h, 64h+32) of the S^T
-          // buffer.
-          auto p_col = [](int k) { return (k < 4) ? k * 8 : 64 + (k - 4) * 8; };
+          // buffer; with dropout the dropped P^T of chunk c (16 queries) in
+          // columns 64h + 16c .. + 7.
+          auto p_col = [](int k) {
+            return DROP ? ((k < 4) ? k * 16 : 64 + (k - 4) * 16) : ((k < 4) ? k * 8 : 64 + (k - 4) * 8);
+          };
           ok = mbar_wait(bar_p_full(buf), (gi / C::NSBUF) & 1, wc);
           if (!ok) break;
           tc_fence_after();
@@ -525,6 +574,12 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         const int s = stg(gi), buf = gi % C::NSBUF;
         const int q0 = (I.qt_begin + it % I.nq) * 128;
         const uint32_t tS = tmem + C::TM_S0 + 128 * buf + lane_off + 64 * half;
+        // dropout: this key's keep bits for the warp's 64 queries, made while
+        // the tensor core computes S^T
+        uint32_t keep[2] = {0u, 0u};
+        if constexpr (DROP)
+          dropout_keep_keyrow_64(keep, key, q0 + 64 * half, (uint32_t)(I.b * p.Hq + I.hkv * G + it / I.nq),
+                                 p.drop_offset, p.seed_lo, p.seed_hi, p.drop_t);
         ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), stg_par(gi), wc));
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(buf), (gi / C::NSBUF) & 1, wc));
         if (!ok) break;
@@ -559,7 +614,18 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             }
             pk[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st8(tS + c * 8, pk);
+          if constexpr (DROP) {
+            // undropped P^T beside the dropped one, both over this chunk's
+            // own (already loaded) S^T columns
+            tmem_st8(tS + c * 16 + 8, pk);
+            const uint32_t kb = keep[c >> 1] >> (16 * (c & 1));
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              pk[e] &= ((kb >> (2 * e)) & 1u ? 0x0000FFFFu : 0u) | ((kb >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u);
+            tmem_st8(tS + c * 16, pk);
+          } else {
+            tmem_st8(tS + c * 8, pk);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -576,7 +642,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off + half * (D / 2);
-        const float mul = which ? p.scale : 1.f;
+        const float mul = which ? p.scale : (DROP ? p.drop_scale : 1.f);
         __nv_bfloat16* dst = (which ? p.dk : p.dv) +
                              (((size_t)I.b * p.Tk + (key < p.Tk ? key : 0)) * p.Hkv + I.hkv) * D + half * (D / 2);
 #pragma unroll
@@ -628,7 +694,25 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         // P^T of this warp's 64 query columns into registers at once, so
         // that the S^T buffer can take the next S^T.
         uint32_t pp[32];
-        tmem_ld32(tP, pp);
+        uint32_t keep[2] = {0u, 0u};
+        if constexpr (DROP) {
+          // undropped P^T, and the keep bits from the dropped copy's zeros
+          // (a kept entry whose P rounds to 0 has dS = 0 either way)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld8(tP + 16 * c + 8, pp + 8 * c);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pd[8];
+            tmem_ld8(tP + 16 * c, pd);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              keep[c >> 1] |= (((pd[e] & 0xFFFFu) != 0u ? 1u : 0u) | ((pd[e] >> 16) != 0u ? 2u : 0u))
+                              << (16 * (c & 1) + 2 * e);
+          }
+        } else {
+          tmem_ld32(tP, pp);
+        }
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar_p_read);
@@ -651,8 +735,17 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           for (int e = 0; e < 8; ++e) {
             const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[8 * c + e]));
             const float2 dd = *reinterpret_cast<const float2*>(drow + 16 * c + 2 * e);
-            const float2 t = __fadd2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
-                                        make_float2(-dd.x, -dd.y));
+            float2 t;
+            if constexpr (DROP) {
+              // Z * s * dP - D
+              const uint32_t kb = keep[c >> 1] >> (16 * (c & 1) + 2 * e);
+              const float2 zs = make_float2(kb & 1u ? p.drop_scale : 0.f, kb & 2u ? p.drop_scale : 0.f);
+              t = __ffma2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])), zs,
+                             make_float2(-dd.x, -dd.y));
+            } else {
+              t = __fadd2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                             make_float2(-dd.x, -dd.y));
+            }
             const float2 r = __fmul2_rn(pf, t);
             pp[8 * c + e] = pack_bf16x2(r.x, r.y);
           }
@@ -764,13 +857,15 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
 }
 
 static int bwd_setup() {
-  const void* kernels[4] = {reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false>),
+  const void* kernels[6] = {reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, true>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false>),
-                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, true>)};
-  const int bytes[4] = {BwdCfg<64>::SMEM_BYTES, BwdCfg<64>::SMEM_BYTES, BwdCfg<128>::SMEM_BYTES,
-                        BwdCfg<128>::SMEM_BYTES};
-  for (int i = 0; i < 4; ++i)
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, true>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false, true>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false, true>)};
+  const int bytes[6] = {BwdCfg<64>::SMEM_BYTES, BwdCfg<64>::SMEM_BYTES, BwdCfg<128>::SMEM_BYTES,
+                        BwdCfg<128>::SMEM_BYTES, BwdCfg<64>::SMEM_BYTES, BwdCfg<128>::SMEM_BYTES};
+  for (int i = 0; i < 6; ++i)
     if (cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes[i]) != cudaSuccess)
       return FA_ERR_CUDA;
   return FA_OK;

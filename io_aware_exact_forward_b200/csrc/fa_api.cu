@@ -95,6 +95,20 @@ static int set_smem(Fn* kernel, int bytes) {
              : FA_ERR_CUDA;
 }
 
+// The forward kernels move registers between warpgroups with setmaxnreg;
+// the split adds up only if the block is launched with exactly the per-thread
+// count it was planned for (an increase beyond the launch's pool would wait
+// forever), so a build that came out differently is refused, not launched.
+template <int D, bool F8, bool DROP>
+static int fwd_setup_one() {
+  using C = FwdCfg<D, F8>;
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, reinterpret_cast<const void*>(fa_fwd_kernel<D, F8, DROP>)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (a.numRegs != C::REG_LAUNCH) return FA_ERR_UNSUPPORTED;
+  return set_smem(fa_fwd_kernel<D, F8, DROP>, C::SMEM_BYTES);
+}
+
 template <int D, int G>
 static int decode_setup_one() {
   int st = set_smem(fa_decode_split_kernel<D, G>, DecCfg<D, G>::SMEM_BYTES);
@@ -123,11 +137,11 @@ static int device_setup_impl() {
     return FA_ERR_CUDA;
   if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
   int st = FA_OK;
-  if (!st) st = set_smem(fa_fwd_kernel<64>, FwdCfg<64>::SMEM_BYTES);
-  if (!st) st = set_smem(fa_fwd_kernel<128>, FwdCfg<128>::SMEM_BYTES);
-  if (!st) st = set_smem(fa_fwd_kernel<128, true>, FwdCfg<128, true>::SMEM_BYTES);
-  if (!st) st = set_smem(fa_fwd_kernel<64, false, true>, FwdCfg<64>::SMEM_BYTES);
-  if (!st) st = set_smem(fa_fwd_kernel<128, false, true>, FwdCfg<128>::SMEM_BYTES);
+  if (!st) st = fwd_setup_one<64, false, false>();
+  if (!st) st = fwd_setup_one<128, false, false>();
+  if (!st) st = fwd_setup_one<128, true, false>();
+  if (!st) st = fwd_setup_one<64, false, true>();
+  if (!st) st = fwd_setup_one<128, false, true>();
   if (!st) st = bwd_setup();
   if (!st) st = decode_setup();
   return st;
@@ -415,9 +429,8 @@ static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO
   p.wait_limit_ns = kWaitLimitNs;
   // Non-causal d = 64: one persistent CTA per SM, whose next item's K/V
   // load overlaps the current item (two K/V buffers); items are all the
-  // same length there.  Otherwise one CTA per item: causal items differ in
-  // length and the hardware scheduler balances them, and at d = 128 there
-  // is room for one K/V buffer only.
+  // same length there.  Causal: one CTA per item, since items differ in
+  // length and the hardware scheduler balances them.
   int nsm = 0;
   if ((st = sm_count(&nsm))) return st;
   const bool persistent = d == 64 && !causal;

@@ -22,14 +22,25 @@
 //               items.
 //   warp 8      MMA issuer (one thread): S_w = Q_w K_j^T into tensor memory,
 //               O_w += P_w V_j with P_w read from tensor memory.
+//   warps 10-11 no role (they complete the third warpgroup, whose registers
+//               go to the softmax warpgroups).
 //   warps 0-3   softmax for query tile 0 (TMEM lanes 0..127, one row per
 //   warps 4-7   thread) and for query tile 1.  Each thread keeps m and l of
 //               its row in registers, writes P (bf16) over its S columns, and
 //               rescales its O row in tensor memory when its reference
 //               maximum moves; then the epilogue writes O = u / l and LSE.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0, O1 after that.
-// The two softmax warpgroups alternate with the tensor core: while one
-// computes exponentials the other's MMAs run.
+// Registers: the block is launched with 168 per thread; the MMA/TMA
+// warpgroup gives all but 72 of them to the two softmax warpgroups (216
+// each), so that a thread holds its whole S row without spilling.  The two
+// softmax warpgroups share each SM sub-partition; per pair of columns the
+// exponentials, the bf16 pack and the two FP32x2 operations cost about 16
+// issue cycles, which bounds the d = 64 kernel.
+//
+// O is normalised by the sum of the P values the P V product actually
+// multiplies (P rounded to bf16), so that O stays a convex combination of
+// V rows however nearly one-hot a row is; LSE uses the sum of the unrounded
+// p.
 //
 // FP8 variant (F8 = true, d = 128): Q, K and V are E4M3 with one dequantising
 // factor per tensor, the two products run as kind::f8f6f4 MMAs (twice the bf16
@@ -96,7 +107,13 @@ struct FwdCfg {
   static constexpr int NBAR = 4 + 2 * NSTAGE + 2 + 2 + 2 + 1 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;
+  // setmaxnreg split of the launch's 384 x 168 registers: two softmax
+  // warpgroups at REG_SOFTMAX, the MMA/TMA warpgroup at REG_OTHER.
+  static constexpr int REG_LAUNCH = 168;
+  static constexpr int REG_SOFTMAX = 216;
+  static constexpr int REG_OTHER = 72;
+  static_assert(128 * (2 * REG_SOFTMAX + REG_OTHER) <= THREADS * REG_LAUNCH, "register split exceeds the launch");
   static constexpr int TMEM_COLS = 512;
   // P apart from S, so that the next S can be computed as soon as the softmax
   // has loaded this one, overlapping the softmax: at d = 64 (bf16) in its own
@@ -110,12 +127,13 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(128, BN, 0, 0) : idesc_bf16_f32(128, BN, 0, 0);
   static constexpr uint32_t IDESC_O = F8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
   static constexpr float RESCALE_THRESHOLD = 8.0f;
-  // Pairs of S columns whose exponentials use exp2_poly2: 3 of every 8 at
-  // d = 128, where the shared MUFU unit limits the softmax, 1 of every 8 at
-  // d = 64 (more costs more FMA-pipe issue than it saves; measured).
-  static constexpr bool poly_pair(int c) {
-    return D == 128 ? ((c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6) : ((c & 7) == 3);
-  }
+  // Pairs of S columns whose exponentials would use exp2_poly2 on the FMA
+  // pipe instead of the MUFU unit.  None: per pair of columns the bf16 pack,
+  // the two FP32x2 sums and the scale cost about as many sub-partition
+  // cycles as the two MUFU exponentials, so moving exponentials to the FMA
+  // pipe slows the softmax at both head sizes (measured 0 < 1/8 < 2/8 < 3/8
+  // of the pairs).
+  static constexpr bool poly_pair(int) { return false; }
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
   static_assert(!F8 || D == 128, "the E4M3 forward is built for d = 128");
 };
@@ -157,7 +175,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
 }
 
 template <int D, bool F8 = false, bool DROP = false>
-__global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -210,8 +228,11 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == 9) {
+  // Each role runs inside the branch that set its register budget, so that
+  // the compiler allocates that budget for it.
+  if (warp >= 8) {
+   setmaxnreg_dec<C::REG_OTHER>();
+   if (warp == 9) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -417,7 +438,9 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
       mma_commit(bar_mma_done);
       mbar_wait_drain(bar_mma_done, 0, p.wait_limit_ns);
     }
+  }
   } else {
+    setmaxnreg_inc<C::REG_SOFTMAX>();
     // ------------------------------------------------------------ softmax
     const int w = warp >> 2;                 // query tile 0 or 1
     const int r = threadIdx.x & 127;         // row within the tile == TMEM lane
@@ -433,7 +456,8 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
       const int key_limit = p.causal ? min(p.Tk, row + (p.Tk - p.Tq) + 1) : p.Tk;  // keys < limit visible
       const int key_lo = p.window > 0 ? row + (p.Tk - p.Tq) - p.window + 1 : 0;     // and keys >= key_lo
       float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
-      float l = 0.f;
+      float l = 0.f;            // sum of the p (the LSE's)
+      float l_r = 0.f;          // sum of the p as rounded for P V (O's normaliser; bf16)
       for (int j = 0; j < it.n_kv; ++j) {
         // dropout: this tile's keep bits, made while the tensor core computes S
         uint32_t keep[4];
@@ -460,16 +484,19 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
           for (int c = 0; c < 128; ++c)
             if (c >= nvalid || c < nlo) su[c] = __float_as_uint(-INFINITY);
         }
-        // Row maximum: eight independent chains, then a short tree.
+        // Row maximum: eight independent chains of three-input maxima (two
+        // new columns per step), then a short tree.
         float mx8[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(su[i]);
+        for (int i = 0; i < 8; ++i) mx8[i] = fmax3(__uint_as_float(su[i]), __uint_as_float(su[8 + i]),
+                                                  __uint_as_float(su[16 + i]));
 #pragma unroll
-        for (int c = 8; c < 128; c += 8)
+        for (int c = 24; c < 120; c += 16)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], __uint_as_float(su[c + i]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], __uint_as_float(su[c + i]), __uint_as_float(su[c + 8 + i]));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], __uint_as_float(su[120 + i]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float m_tile = mx * p.scale_log2;
         // Lazy rescale: move the reference only when the maximum grew by more
         // than the threshold (or there was no reference yet).
@@ -479,11 +506,23 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
           alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_tile);
           m_ref = m_tile;
           l *= alpha;
+          l_r *= alpha;
         }
         const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
         const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nref = make_float2(-ref, -ref);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 acc_r[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        if constexpr (C::SEP_P && !F8) {
+          // P's columns are free once the previous tile's PV completed
+          // (normally long since): P is stored in two halves as the loop
+          // below produces it
+          if (g + j > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_p_free(w), (g + j - 1) & 1, wc));
+            if (!ok) break;
+          }
+          tc_fence_after();
+        }
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(su[2 * c]), __uint_as_float(su[2 * c + 1])), sl2, nref);
@@ -495,29 +534,44 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
             if (2 * c + 1 >= nvalid || 2 * c + 1 < nlo) pr.y = 0.f;
           }
           acc[c & 3] = __fadd2_rn(acc[c & 3], pr);   // l sums the undropped p
-          if constexpr (DROP) {
-            const uint32_t kb = keep[c >> 4] >> ((2 * c) & 31);
-            pr.x = (kb & 1u) ? pr.x : 0.f;
-            pr.y = (kb & 2u) ? pr.y : 0.f;
-          }
           if constexpr (F8) {
+            if constexpr (DROP) {
+              const uint32_t kb = keep[c >> 4] >> ((2 * c) & 31);
+              pr.x = (kb & 1u) ? pr.x : 0.f;
+              pr.y = (kb & 2u) ? pr.y : 0.f;
+            }
             // four E4M3 values per column; su[c >> 1] was consumed at step c >> 2
             const uint32_t h = pack_e4m3x2(pr.x, pr.y);
             su[c >> 1] = (c & 1) ? (su[c >> 1] | (h << 16)) : h;
           } else {
-            su[c] = pack_bf16x2(pr.x, pr.y);
+            uint32_t pk = pack_bf16x2(pr.x, pr.y);
+            // l_r sums the undropped p as rounded (bf16 to fp32 is a shift)
+            acc_r[c & 1] = __fadd2_rn(acc_r[c & 1], make_float2(__uint_as_float(pk << 16),
+                                                                 __uint_as_float(pk & 0xFFFF0000u)));
+            if constexpr (DROP) {
+              const uint32_t kb = keep[c >> 4] >> ((2 * c) & 31);
+              pk &= ((kb & 1u) ? 0x0000FFFFu : 0u) | ((kb & 2u) ? 0xFFFF0000u : 0u);
+            }
+            su[c] = pk;
+            // each half of P (32 columns) goes to tensor memory while the
+            // next half is computed: P's own columns (d = 64) or, at d = 128,
+            // the S columns already in registers
+            if (c == 31 || c == 63) tmem_st32((C::SEP_P ? tP : tS) + (c == 63 ? 32 : 0), su + (c == 63 ? 32 : 0));
           }
         }
         const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
         l += a.x + a.y;
-        if constexpr (C::SEP_P) {
-          // P's columns and O are free once the previous tile's PV completed
+        const float2 ar = __fadd2_rn(acc_r[0], acc_r[1]);
+        l_r += ar.x + ar.y;
+        if constexpr (F8) {
+          // P's shared-memory tile and O are free once the previous tile's
+          // PV completed
           if (g + j > 0) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar_p_free(w), (g + j - 1) & 1, wc));
             if (!ok) break;
           }
           tc_fence_after();
-          if constexpr (F8) {
+          {
             // row r of P_w: eight 16-byte chunks, chunk c stored at c ^ (r & 7)
             // (the 128-byte swizzle the MMA's descriptor names)
             uint8_t* prow = smem + C::OFF_P + w * C::P_BYTES + r * 128;
@@ -526,13 +580,7 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
               *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
                   make_uint4(su[4 * c], su[4 * c + 1], su[4 * c + 2], su[4 * c + 3]);
             fence_proxy_async_smem();
-          } else {
-            tmem_st32(tP, su);
-            tmem_st32(tP + 32, su + 32);
           }
-        } else {
-          tmem_st32(tS, su);
-          if constexpr (!F8) tmem_st32(tS + 32, su + 32);
         }
         if (j > 0 && __any_sync(0xffffffffu, move)) {
           // O row *= alpha.  The PV of the previous tile has completed (with
@@ -561,7 +609,8 @@ __global__ void __launch_bounds__(320, 1) fa_fwd_kernel(const __grid_constant__ 
         tc_fence_after();
       }
       const bool in_range = row < p.Tq;
-      const float inv_l = (l > 0.f) ? p.o_scale / l : 0.f;
+      const float l_o = F8 ? l : l_r;
+      const float inv_l = (l_o > 0.f) ? p.o_scale / l_o : 0.f;
       __nv_bfloat16* orow = p.o + (((size_t)it.b * p.Tq + (in_range ? row : 0)) * p.Hq + it.h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

@@ -268,12 +268,13 @@ static int forward_impl(const void* q, const void* k, const void* v, void* o, fl
   p.n_mblocks = (Tq + 255) / 256;
   p.n_items = B * Hq * p.n_mblocks;
   p.wait_limit_ns = kWaitLimitNs;
-  // Uniform (non-causal) items: persistent, one CTA per SM.  Causal items
-  // differ in cost: one CTA per item, heaviest first, balanced by the block
-  // scheduler.
+  // Uniform (non-causal or sliding-window) items: persistent, one CTA per
+  // SM.  Causal items differ in cost: one CTA per item, heaviest first,
+  // balanced by the block scheduler.
   int nsm = 0;
   if ((st = sm_count(&nsm))) return st;
-  dim3 grid(causal ? p.n_items : std::min(p.n_items, nsm));
+  // Sliding-window items are about equally long: persistent as well.
+  dim3 grid(causal && window == 0 ? p.n_items : std::min(p.n_items, nsm));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (f8)
     fa_fwd_kernel<128, true><<<grid, FwdCfg<128, true>::THREADS, FwdCfg<128, true>::SMEM_BYTES, s>>>(p);

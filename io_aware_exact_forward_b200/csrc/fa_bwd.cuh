@@ -319,7 +319,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
   const uint32_t bar_do_full = bar0 + 8u * 23;   // single dO buffer (d = 128)
   const uint32_t bar_p_read = bar0 + 8u * 24;    // the dS warps hold this tile's P^T
   const uint32_t bar_do_empty = bar0 + 8u * 25;
-  const uint32_t bar_ds_free = bar0 + 8u * 26;   // the tile's dK and dQ have read the dS tile
+  const uint32_t bar_ds_free = bar0 + 8u * 26;   // d = 64: the tile's dQ and dK have read the dS tile
   // Q/dO stage of global iteration g and the parity of its use of that stage.
   auto stg = [&](int g) { return g % C::NQ; };
   auto stg_par = [&](int g) { return (uint32_t)((g / C::NQ) & 1); };
@@ -462,27 +462,17 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         const BwdItem I = bwd_item(p, item);
         if (I.n_it == 0) continue;
         const int kvb = ki % C::NKV;
-        // The first S^T and dP^T of an item: issued here for the CTA's first
-        // item, and for every item with a single K/V buffer (d = 128), whose
-        // next item's K and V can only load once this item's last dQ has read
-        // K; with two K/V buffers they are issued ahead by the item before.
-        if (!started || C::NKV == 1) {
-          if (started) {
-            // S^T over the last tile's P^T (loaded by the dS warps) and dP^T
-            // over its dQ (read out)
-            ok = mbar_wait(bar_p_read, (gi - 1) & 1, wc);
-            if (ok) ok = mbar_wait(bar_dq_free(0), (gi - 1) & 1, wc);
-          }
-          if (ok) ok = mbar_wait(bar_kv_full(kvb), (ki / C::NKV) & 1, wc);
-          if (ok) ok = mbar_wait(bar_qdo_full(stg(gi)), stg_par(gi), wc);
-          if (ok) ok = wait_do(gi);
+        if (!started) {
+          ok = mbar_wait(bar_kv_full(kvb), (ki / C::NKV) & 1, wc);
+          if (ok) ok = mbar_wait(bar_qdo_full(stg(0)), stg_par(0), wc);
+          if (ok) ok = wait_do(0);
           if (!ok) break;
           tc_fence_after();
-          issue_s(gi, kvb);
-          issue_dp(gi, kvb);
+          issue_s(0, kvb);
+          issue_dp(0, kvb);
           started = true;
         }
-        const bool has_next_item = C::NKV > 1 && item + (int)gridDim.x < p.n_items;
+        const bool has_next_item = item + (int)gridDim.x < p.n_items;
         for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
           const int buf = gi % C::NSBUF;
           const bool last = it + 1 == I.n_it;
@@ -536,35 +526,35 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           ok = mbar_wait(bar_ds_full, gi & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          // dQ = dS K: with two S^T buffers into this tile's (P^T was read
-          // above); with one, into the dP^T columns, which the dS warps have
-          // read (the S^T buffer already holds the next S^T).
           // dK += dS^T Q with dS^T read from the shared dS tile (key rows,
           // query columns: K-major for this product); its completion frees
-          // the Q stage.  At d = 64 dQ goes first, so that its read-out,
-          // which the next-but-one S^T waits for, starts one product earlier
-          // (measured 6% faster); at d = 128 dK first measured faster.
-          // The second of the two frees the dS tile.
+          // the Q stage.  dQ = dS K: with two S^T buffers (d = 64) into this
+          // tile's (P^T was read above); with one (d = 128), into the dP^T
+          // columns, which the dS warps have read (the S^T buffer already
+          // holds the next S^T).  At d = 64 dQ goes first, so that its
+          // read-out, which the next-but-one S^T waits for, starts one
+          // product earlier (measured 6% faster), and a separate commit
+          // after dK frees the dS tile; at d = 128 dK first measured faster,
+          // and dQ's completion frees the tile.
           const uint32_t tDQ = C::NSBUF == 1 ? tDP : tS(buf);
-          auto issue_dq = [&]() {
+          if constexpr (D == 64) {
 #pragma unroll
             for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
             mma_commit(bar_dq_full(buf));
-          };
-          auto issue_dk = [&]() {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               mma_ss(tDK, kdesc(aDS, k), mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
             mma_commit(bar_qdo_empty(stg(gi)));
-          };
-          if (D == 64) {
-            issue_dq();
-            issue_dk();
+            mma_commit(bar_ds_free);
           } else {
-            issue_dk();
-            issue_dq();
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              mma_ss(tDK, kdesc(aDS, k), mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
+            mma_commit(bar_qdo_empty(stg(gi)));
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
+            mma_commit(bar_dq_full(buf));
           }
-          mma_commit(bar_ds_free);
           if (last) {
             mma_commit(bar_kv_empty(kvb));
             mma_commit(bar_dkdv_done);
@@ -777,9 +767,11 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           }
           if (c == 0 && gi > 0) {
             // The shared dS tile is still an operand of the previous tile's
-            // dQ and dK MMAs until they complete (this tile's dP^T can
+            // dK and dQ MMAs until they complete (this tile's dP^T can
             // complete before them).
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_ds_free, (gi - 1) & 1, wc));
+            ok = __all_sync(0xffffffffu,
+                            D == 64 ? mbar_wait(bar_ds_free, (gi - 1) & 1, wc)
+                                    : mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
             if (!ok) break;
           }
           // dS into shared memory: row j of box `half`, 16-byte chunks 2c and
@@ -818,8 +810,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         // Passes of BPP 32-column boxes: TMEM loads, then staging and bulk
         // reduce-adds; the columns are released after the last pass's
         // loads.  d = 64 takes one box per pass (fewer live registers, no
-        // spills: measured faster than two); d = 128 two, which releases its
-        // four boxes sooner.
+        // spills); d = 128 two, which releases its four boxes sooner.
         constexpr int BPP = (D == 64) ? 1 : 2;
 #pragma unroll
         for (int pr = 0; pr < D / 32 / BPP; ++pr) {

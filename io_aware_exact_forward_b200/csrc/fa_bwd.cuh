@@ -438,11 +438,14 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
       auto aQ = [&](int g) { return sbase + C::OFF_Q + stg(g) * C::TILE; };
       auto aDO = [&](int g) { return sbase + C::OFF_DO + (C::SPLIT_DO ? 0 : stg(g) * C::TILE); };
       auto wait_do = [&](int g) { return !C::SPLIT_DO || mbar_wait(bar_do_full, g & 1, wc); };
+      // Descriptors: the low word of the tile's first slice plus the slice
+      // offset / 16 (the tile's low word is common to the unrolled slices).
+      constexpr uint32_t HI = sw128_hi(1024);
       auto kdesc = [&](uint32_t base, int k) {  // K-major tile, k-th 16-element slice of d
-        return smem_desc_sw128(base + (k >> 2) * C::BOX_BYTES + (k & 3) * 32, 16, 1024);
+        return sw128_desc(sw128_lo(base, 16) + (((k >> 2) * C::BOX_BYTES + (k & 3) * 32) >> 4), HI);
       };
       auto mndesc = [&](uint32_t base, int k) {  // MN-major view, k-th 16-row slice
-        return smem_desc_sw128(base + k * 16 * 128, C::BOX_BYTES, 1024);
+        return sw128_desc(sw128_lo(base, C::BOX_BYTES) + ((k * 16 * 128) >> 4), HI);
       };
       auto issue_s = [&](int g, int kvb) {
         const int buf = g % C::NSBUF;

@@ -301,11 +301,15 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
     if (lane == 0) {
       const uint32_t tS[2] = {tmem, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      // Descriptors: the low word of the tile's first K slice plus the slice
+      // offset / 16 (the high word is the same for every operand here).
+      constexpr uint32_t HI = sw128_hi(1024);
       auto issue_s = [&](int w, uint32_t qa, int sK) {
+        const uint32_t a0 = sw128_lo(qa, 16), b0 = sw128_lo(stage_addr(sK), 16);
 #pragma unroll
         for (int k = 0; k < D / C::KSTEP; ++k) {
-          const uint32_t off = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;
-          const uint64_t da = smem_desc_sw128(qa + off, 16, 1024), db = smem_desc_sw128(stage_addr(sK) + off, 16, 1024);
+          const uint32_t o = ((k >> 2) * C::BOX_BYTES + (k & 3) * 32) >> 4;
+          const uint64_t da = sw128_desc(a0 + o, HI), db = sw128_desc(b0 + o, HI);
           if constexpr (F8) mma_ss_f8(tS[w], da, db, C::IDESC_S, k > 0);
           else mma_ss(tS[w], da, db, C::IDESC_S, k > 0);
         }
@@ -313,9 +317,10 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
       // P (over S's first columns) times V_j: each MMA takes KSTEP keys, 32
       // bytes of P per row (8 columns) and KSTEP rows of the V tile.
       auto issue_pv = [&](int w, int sV, bool first) {
+        const uint32_t v0 = sw128_lo(stage_addr(sV), C::BOX_BYTES);
 #pragma unroll
         for (int k = 0; k < C::BN / C::KSTEP; ++k) {
-          const uint64_t db = smem_desc_sw128(stage_addr(sV) + k * C::KSTEP * 128, C::BOX_BYTES, 1024);
+          const uint64_t db = sw128_desc(v0 + ((k * C::KSTEP * 128) >> 4), HI);
           if constexpr (F8) mma_ts_f8(tO[w], tS[w] + k * 8, db, C::IDESC_O, (!first) || k > 0);
           else mma_ts(tO[w], tS[w] + k * 8, db, C::IDESC_O, (!first) || k > 0);
         }
@@ -329,12 +334,14 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
         // commits p_free, which releases the P columns and O to the softmax.
         const uint32_t tP[2] = {tmem + C::TM_P, tmem + C::TM_P + 64};
         auto issue_pv_p = [&](int w, int sV, bool first) {
+          const uint32_t v0 = sw128_lo(stage_addr(sV), C::BOX_BYTES);
+          const uint32_t p0 = sw128_lo(sbase + C::OFF_P + w * C::P_BYTES, 16);
 #pragma unroll
           for (int k = 0; k < C::BN / C::KSTEP; ++k) {
-            const uint64_t db = smem_desc_sw128(stage_addr(sV) + k * C::KSTEP * 128, C::BOX_BYTES, 1024);
+            const uint64_t db = sw128_desc(v0 + ((k * C::KSTEP * 128) >> 4), HI);
             if constexpr (F8) {
               // P_w in shared memory: K-major, 128-byte rows, 128-byte swizzle
-              const uint64_t da = smem_desc_sw128(sbase + C::OFF_P + w * C::P_BYTES + k * 32, 16, 1024);
+              const uint64_t da = sw128_desc(p0 + ((k * 32) >> 4), HI);
               mma_ss_f8(tO[w], da, db, C::IDESC_O, (!first) || k > 0);
             } else {
               mma_ts(tO[w], tP[w] + k * 8, db, C::IDESC_O, (!first) || k > 0);
@@ -513,10 +520,12 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
         const float2 nref = make_float2(-ref, -ref);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         float2 acc_r[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        if constexpr (C::SEP_P && !F8) {
-          // P's columns are free once the previous tile's PV completed
-          // (normally long since): P is stored in two halves as the loop
-          // below produces it
+        if constexpr (C::SEP_P) {
+          // P's columns (E4M3: P's shared-memory tile) and O are free once
+          // the previous tile's PV completed (normally long since): bf16 P is
+          // stored in two halves as the loop below produces it.  Waiting here
+          // rather than after the loop measured 12% faster for E4M3 (1444
+          // against 1292 TFLOP/s on the 32k causal GQA workload).
           if (g + j > 0) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar_p_free(w), (g + j - 1) & 1, wc));
             if (!ok) break;
@@ -564,13 +573,6 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
         const float2 ar = __fadd2_rn(acc_r[0], acc_r[1]);
         l_r += ar.x + ar.y;
         if constexpr (F8) {
-          // P's shared-memory tile and O are free once the previous tile's
-          // PV completed
-          if (g + j > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_p_free(w), (g + j - 1) & 1, wc));
-            if (!ok) break;
-          }
-          tc_fence_after();
           {
             // row r of P_w: eight 16-byte chunks, chunk c stored at c ^ (r & 7)
             // (the 128-byte swizzle the MMA's descriptor names)

@@ -306,15 +306,27 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 //   lbo:   leading byte offset (MN-major: stride between 64-element column
 //          blocks; unused for K-major swizzled layouts)
 //   sbo:   stride byte offset (stride between consecutive 8-row groups)
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t start, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((start >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1u << 46;   // descriptor version for tcgen05
-  d |= (uint64_t)2u << 61;   // layout: 128-byte swizzle
-  return d;
+// The descriptor as two 32-bit words.  Low: start (bits 0-13, 16-byte
+// units) and lbo (bits 16-29).  High: sbo (bits 0-13), the version (bit 14)
+// and the layout (bits 29-31: 2 = 128-byte swizzle).
+__device__ __forceinline__ uint32_t sw128_lo(uint32_t start, uint32_t lbo) {
+  return ((start >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
 }
+__host__ __device__ constexpr uint32_t sw128_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t lo, uint32_t hi) {
+  return ((uint64_t)hi << 32) | lo;
+}
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  return sw128_desc(sw128_lo(start, lbo), sw128_hi(sbo));
+}
+// The MMA loops keep the low word of an operand's first K slice and add the
+// slice's byte offset / 16: one integer add per MMA instead of rebuilding the
+// descriptor.  The MMA-issuing thread shares its sub-partition with busy
+// softmax warps, so its instruction count sets how fast it can feed the
+// tensor core.  (Shared-memory addresses stay below 2^18 bytes, so the
+// 14-bit start field never carries into the lbo field.)
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 //   a_mn / b_mn: 1 if that operand is MN-major (transposed) in shared memory.

@@ -278,8 +278,7 @@ __device__ __forceinline__ void dropout_keep_keyrow_64(uint32_t (&mask)[2], int 
       const int want = (q - s) & 3;      // the key (quad-mate) this lane sends to
       const uint32_t send = want == 0 ? x[0] : want == 1 ? x[1] : want == 2 ? x[2] : x[3];
       const uint32_t got = s == 0 ? send : __shfl_sync(0xffffffffu, send, (lane & ~3) | src);
-      const uint32_t lt = __vcmpltu4(got, tt);   // 0xFF in each byte below t
-      const uint32_t bits = ((lt >> 7) & 1u) | ((lt >> 14) & 2u) | ((lt >> 21) & 4u) | ((lt >> 28) & 8u);
+      const uint32_t bits = gather_msb4(bytes_below(got, tt));  // bit j: byte j below t
       // queries 4 (4m + src) .. + 3 of the 64: word m / 2, bits 16 (m & 1) + 4 src
       mask[m >> 1] |= bits << (16 * (m & 1) + 4 * src);
     }

@@ -412,12 +412,27 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
       k0 += kW0;
       k1 += kW1;
     }
-    const uint32_t hi0 = __umulhi(kM0, c.x), lo0 = kM0 * c.x;
-    const uint32_t hi1 = __umulhi(kM1, c.z), lo1 = kM1 * c.z;
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    // one 32 x 32 -> 64-bit product per multiplier gives both halves
+    const uint64_t p0 = (uint64_t)kM0 * c.x, p1 = (uint64_t)kM1 * c.z;
+    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1, (uint32_t)p0);
   }
   return c;
 }
+
+// Bit 7 of each byte of the result is set iff that byte of b is below t
+// (every byte of tt is t; the other bits are zero).  Per byte, with the top
+// bits set aside, (b | 0x80) - (t & 0x7F) cannot borrow from the next byte
+// and its bit 7 says (b & 0x7F) >= (t & 0x7F); then b < t iff b7 < t7, or
+// b7 == t7 and the low seven bits are below.
+__device__ __forceinline__ uint32_t bytes_below(uint32_t b, uint32_t tt) {
+  const uint32_t x = (b | 0x80808080u) - (tt & 0x7F7F7F7Fu);
+  return ((~b & tt) | (~(b ^ tt) & ~x)) & 0x80808080u;
+}
+
+// Bits 7, 15, 23 and 31 of m (all other bits zero) as bits 0..3: the
+// product puts each at bit 28 + its byte, and no two partial products share
+// a bit.
+__device__ __forceinline__ uint32_t gather_msb4(uint32_t m) { return (m * 0x00204081u) >> 28; }
 
 // Keep bits of query row `row` for the 128 keys key0 .. key0 + 127 (key0 a
 // multiple of 16): bit k of mask[k >> 5] is key key0 + k.  The block of rows
@@ -442,8 +457,7 @@ __device__ __forceinline__ void dropout_keep_128(uint32_t (&mask)[4], int row, i
       const int want = (q - s) & 3;      // the word the receiving lane needs
       const uint32_t send = want == 0 ? wv.x : want == 1 ? wv.y : want == 2 ? wv.z : wv.w;
       const uint32_t got = s == 0 ? send : __shfl_sync(0xffffffffu, send, (lane & ~3) | src);
-      const uint32_t lt = __vcmpltu4(got, tt);   // 0xFF in each byte below t
-      const uint32_t bits = ((lt >> 7) & 1u) | ((lt >> 14) & 2u) | ((lt >> 21) & 4u) | ((lt >> 28) & 8u);
+      const uint32_t bits = gather_msb4(bytes_below(got, tt));  // bit j: byte j below t
       // keys 4 * (4m + src) .. + 3 of the tile: word m / 2, bits 16 (m & 1) + 4 src
       mask[m >> 1] |= bits << (16 * (m & 1) + 4 * src);
     }

@@ -101,7 +101,7 @@ static int set_smem(Fn* kernel, int bytes) {
 // forever), so a build that came out differently is refused, not launched.
 template <int D, bool F8, bool DROP>
 static int fwd_setup_one() {
-  using C = FwdCfg<D, F8>;
+  using C = FwdCfg<D, F8, DROP>;
   cudaFuncAttributes a;
   if (cudaFuncGetAttributes(&a, reinterpret_cast<const void*>(fa_fwd_kernel<D, F8, DROP>)) != cudaSuccess)
     return FA_ERR_CUDA;
@@ -279,9 +279,9 @@ static int forward_impl(const void* q, const void* k, const void* v, void* o, fl
   if (f8)
     fa_fwd_kernel<128, true><<<grid, FwdCfg<128, true>::THREADS, FwdCfg<128, true>::SMEM_BYTES, s>>>(p);
   else if (drop && d == 64)
-    fa_fwd_kernel<64, false, true><<<grid, FwdCfg<64>::THREADS, FwdCfg<64>::SMEM_BYTES, s>>>(p);
+    fa_fwd_kernel<64, false, true><<<grid, FwdCfg<64, false, true>::THREADS, FwdCfg<64, false, true>::SMEM_BYTES, s>>>(p);
   else if (drop)
-    fa_fwd_kernel<128, false, true><<<grid, FwdCfg<128>::THREADS, FwdCfg<128>::SMEM_BYTES, s>>>(p);
+    fa_fwd_kernel<128, false, true><<<grid, FwdCfg<128, false, true>::THREADS, FwdCfg<128, false, true>::SMEM_BYTES, s>>>(p);
   else if (d == 64)
     fa_fwd_kernel<64><<<grid, FwdCfg<64>::THREADS, FwdCfg<64>::SMEM_BYTES, s>>>(p);
   else

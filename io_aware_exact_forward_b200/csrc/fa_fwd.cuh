@@ -23,7 +23,8 @@
 //   warp 8      MMA issuer (one thread): S_w = Q_w K_j^T into tensor memory,
 //               O_w += P_w V_j with P_w read from tensor memory.
 //   warps 10-11 no role (they complete the third warpgroup, whose registers
-//               go to the softmax warpgroups).
+//               go to the softmax warpgroups), except with dropout at d = 64,
+//               where they make each KV tile's keep bits for the softmax.
 //   warps 0-3   softmax for query tile 0 (TMEM lanes 0..127, one row per
 //   warps 4-7   thread) and for query tile 1.  Each thread keeps m and l of
 //               its row in registers, writes P (bf16) over its S columns, and
@@ -54,8 +55,10 @@
 // Dropout variant (DROP = true, bf16): P is multiplied by a keep mask before
 // P V ("Efficient attention: memory-bound", "Real code moves even more", puts
 // dropout on the probabilities before the final product); the mask is
-// regenerated from Philox-4x32-10 for each tile, l sums the undropped P, and
-// the epilogue scales O by 256 / t.
+// regenerated from Philox-4x32-10 for each tile (at d = 64 by warps 10-11,
+// which otherwise have no role, into shared memory; at d = 128 by the
+// softmax threads themselves), l sums the undropped P, and the epilogue
+// scales O by 256 / t.
 //
 // The rescale is lazy: a row keeps its reference maximum until the running
 // maximum exceeds it by more than 8 (log2 units), so exponentials stay below
@@ -85,7 +88,7 @@ struct FwdParams {
   unsigned long long wait_limit_ns;
 };
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool DROP = false>
 struct FwdCfg {
   static constexpr int BM = 128;                 // rows per query tile
   static constexpr int BN = 128;                 // keys per KV tile
@@ -101,10 +104,19 @@ struct FwdCfg {
   // E4M3: P0, P1 (128 rows x 128 one-byte keys each) in shared memory
   static constexpr int P_BYTES = BM * BN;
   static constexpr int OFF_P = OFF_RING + NSTAGE * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_P + (F8 ? 2 * P_BYTES : 0);
+  // Dropout at d = 64: warps 10-11 (otherwise without a role) make each KV
+  // tile's keep bits ahead of the softmax, into two buffers of
+  // [2 query tiles][128 rows] x 128 bits; the softmax threads load their
+  // row's 16 bytes.  (At d = 128 shared memory is full and the softmax
+  // threads make their own.)
+  static constexpr bool MASKW = DROP && D == 64 && !F8;
+  static constexpr int OFF_MASK = OFF_P + (F8 ? 2 * P_BYTES : 0);
+  static constexpr int MASK_BYTES = MASKW ? 2 * 2 * 128 * 16 : 0;
+  static constexpr int OFF_BAR = OFF_MASK + MASK_BYTES;
   // q_full[2], q_empty[2], kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2],
-  // p_full[2], o_final[2], mma_done, s_free[2], p_free[2]
-  static constexpr int NBAR = 4 + 2 * NSTAGE + 2 + 2 + 2 + 1 + 4;
+  // p_full[2], o_final[2], mma_done, s_free[2], p_free[2] (, mask_full[2],
+  // mask_empty[2])
+  static constexpr int NBAR = 4 + 2 * NSTAGE + 2 + 2 + 2 + 1 + 4 + (MASKW ? 4 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
@@ -176,7 +188,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
 
 template <int D, bool F8 = false, bool DROP = false>
 __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<D, F8>;
+  using C = FwdCfg<D, F8, DROP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -191,6 +203,9 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
   const uint32_t bar_mma_done = bar_base + 8u * (10 + 2 * C::NSTAGE);
   auto bar_s_free = [&](int w) { return bar_base + 8u * (11 + 2 * C::NSTAGE + w); };  // softmax loaded S
   auto bar_p_free = [&](int w) { return bar_base + 8u * (13 + 2 * C::NSTAGE + w); };  // PV read P, wrote O
+  // dropout keep bits of KV tile t in buffer t & 1: written / read by every row
+  auto bar_mask_full = [&](int b) { return bar_base + 8u * (15 + 2 * C::NSTAGE + b); };
+  auto bar_mask_empty = [&](int b) { return bar_base + 8u * (17 + 2 * C::NSTAGE + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   auto q_addr = [&](int qb, int w) { return sbase + C::OFF_Q + (2 * qb + w) * C::TILE_BYTES; };
@@ -216,6 +231,10 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
       mbar_init(bar_o_final(w), 1);
       mbar_init(bar_s_free(w), 128);
       mbar_init(bar_p_free(w), 1);
+      if (C::MASKW) {
+        mbar_init(bar_mask_full(w), 64);
+        mbar_init(bar_mask_empty(w), 256);
+      }
     }
     mbar_init(bar_mma_done, 1);
     fence_barrier_init();
@@ -295,6 +314,49 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
             mbar_wait_drain(bar_kv_full(k % C::NSTAGE), (k / C::NSTAGE) & 1, p.wait_limit_ns);
         }
       }
+    }
+  } else if (C::MASKW && warp >= 10) {
+    // ------------------------------------------------------------ dropout mask
+    // Thread mt makes rows 4 (mt & 31) .. + 3 of query tile mt >> 5: for each
+    // of the tile's 32 key groups the Philox block of those four rows (the
+    // layout the softmax's own generator uses: counter (row / 4, key / 4, bh,
+    // offset), word = row, byte = key), each row's keep bits gathered into
+    // its four 32-key words.
+    const int mt = threadIdx.x - 320;
+    const int wq = mt >> 5, a_loc = mt & 31;
+    const uint32_t tt = p.drop_t * 0x01010101u;
+    uint4* mbuf = reinterpret_cast<uint4*>(smem + C::OFF_MASK);
+    bool ok = true;
+    int g = 0;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const FwdItem it = fwd_item<D>(p, item);
+      if (it.n_kv == 0) continue;
+      const uint32_t a_glob = (uint32_t)((it.m0 + wq * C::BM) >> 2) + (uint32_t)a_loc;
+      const uint32_t bh = (uint32_t)(it.b * p.Hq + it.h);
+      for (int j = 0; j < it.n_kv && ok; ++j) {
+        const int t = g + j, buf = t & 1;
+        if (t >= 2) ok = mbar_wait(bar_mask_empty(buf), ((t >> 1) - 1) & 1, wc);
+        if (!ok) break;
+        const uint32_t c0 = (uint32_t)((it.kv0 + j) * C::BN) >> 2;
+        uint32_t* mw = reinterpret_cast<uint32_t*>(mbuf + (buf * 2 + wq) * 128 + 4 * a_loc);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {  // keys 32k .. 32k + 31: eight Philox blocks
+          uint32_t rw[4] = {0u, 0u, 0u, 0u};  // one word per row of the group
+#pragma unroll
+          for (int cl = 8 * k; cl < 8 * k + 8; ++cl) {
+            const uint4 v = philox4x32_10(make_uint4(a_glob, c0 + cl, bh, p.drop_offset), p.seed_lo, p.seed_hi);
+            const int sh = 4 * (cl & 7);
+            rw[0] |= gather_msb4(bytes_below(v.x, tt)) << sh;
+            rw[1] |= gather_msb4(bytes_below(v.y, tt)) << sh;
+            rw[2] |= gather_msb4(bytes_below(v.z, tt)) << sh;
+            rw[3] |= gather_msb4(bytes_below(v.w, tt)) << sh;
+          }
+#pragma unroll
+          for (int w4 = 0; w4 < 4; ++w4) mw[4 * w4 + k] = rw[w4];
+        }
+        mbar_arrive(bar_mask_full(buf));
+      }
+      g += it.n_kv;
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
@@ -468,9 +530,21 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
       for (int j = 0; j < it.n_kv; ++j) {
         // dropout: this tile's keep bits, made while the tensor core computes S
         uint32_t keep[4];
-        if constexpr (DROP)
+        if constexpr (C::MASKW) {
+          // this row's keep bits from the mask warps
+          const int t = g + j, mb = t & 1;
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_mask_full(mb), (t >> 1) & 1, wc));
+          if (!ok) break;
+          const uint4 kv = reinterpret_cast<const uint4*>(smem + C::OFF_MASK)[(mb * 2 + w) * 128 + r];
+          keep[0] = kv.x;
+          keep[1] = kv.y;
+          keep[2] = kv.z;
+          keep[3] = kv.w;
+          mbar_arrive(bar_mask_empty(mb));
+        } else if constexpr (DROP) {
           dropout_keep_128(keep, row, (it.kv0 + j) * C::BN, (uint32_t)(it.b * p.Hq + it.h), p.drop_offset,
                            p.seed_lo, p.seed_hi, p.drop_t);
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(w), (g + j) & 1, wc));
         if (!ok) break;
         tc_fence_after();

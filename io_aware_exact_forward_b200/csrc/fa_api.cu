@@ -440,9 +440,9 @@ static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO
   if (drop && window > 0) return FA_ERR_UNSUPPORTED;
   if (drop) {
     if (d == 64)
-      fa_bwd_dkdv_kernel<64, false, true><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+      fa_bwd_dkdv_kernel<64, false, true><<<grid, BwdCfg<64, true>::THREADS, BwdCfg<64, true>::SMEM_BYTES, s>>>(p);
     else
-      fa_bwd_dkdv_kernel<128, false, true><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+      fa_bwd_dkdv_kernel<128, false, true><<<grid, BwdCfg<128, true>::THREADS, BwdCfg<128, true>::SMEM_BYTES, s>>>(p);
   } else if (d == 64) {
     if (window > 0)
       fa_bwd_dkdv_kernel<64, true><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);

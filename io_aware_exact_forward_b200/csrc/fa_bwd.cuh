@@ -40,7 +40,7 @@
 // Warp roles in dkdv: 0-7 P^T and, at an item's end, dK/dV out; 8-15 dS
 // (two warps per TMEM lane quarter, one per half of the 128 query columns);
 // 16-19 dQ read-out and reduce-adds (one query row per thread); 20 MMA
-// issuer; 21 TMA producer.
+// issuer; 21 TMA producer; with dropout at d = 64, 22-23 make the keep bits.
 #pragma once
 
 #include "fa_ptx.cuh"
@@ -162,7 +162,7 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 }
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-template <int D>
+template <int D, bool DROP = false>
 struct BwdCfg {
   static constexpr int NBOX = D / 64;
   static constexpr int BOX_BYTES = 128 * 128;
@@ -191,16 +191,23 @@ struct BwdCfg {
   static constexpr int DQS_BYTES = NDQS * 128 * 32 * 4;
   static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;   // [NQ][128] f32
   static constexpr int OFF_DD = OFF_LSE + NQ * 128 * 4; // [NQ][128] f32
-  static constexpr int OFF_BAR = OFF_DD + NQ * 128 * 4;
+  // Dropout at d = 64: warps 22-23 make each query tile's keep bits ahead
+  // of the P^T warps, into two buffers of [128 keys][2 query halves] x 64
+  // bits; the P^T warps load their key's 8 bytes.  (At d = 128 shared
+  // memory is full and the P^T warps make their own.)
+  static constexpr bool MASKW = DROP && D == 64;
+  static constexpr int OFF_MASK = OFF_DD + NQ * 128 * 4;
+  static constexpr int MASK_BYTES = MASKW ? 2 * 128 * 2 * 8 : 0;
+  static constexpr int OFF_BAR = OFF_MASK + MASK_BYTES;
   // kv_full[2], kv_empty[2], qdo_full[3], qdo_empty[3], s_full[2], p_full[2],
   // dp_full, ds_full, dq_full[2], dq_free[2], dkdv_done, mma_done, dp_free,
-  // do_full, p_read, do_empty, ds_free
-  static constexpr int NBAR = 27;
+  // do_full, p_read, do_empty, ds_free (, mask_full[2], mask_empty[2])
+  static constexpr int NBAR = 27 + (MASKW ? 4 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   // warps 0-7 P^T (two per TMEM lane quarter, one per half of the query
   // columns), 8-15 dS, 16-19 dQ, 20 MMA issuer, 21 TMA producer
-  static constexpr int THREADS = 704;
+  static constexpr int THREADS = MASKW ? 768 : 704;
   static constexpr int MMA_WARP = 20;
   static constexpr int LOAD_WARP = 21;
   static constexpr int TMEM_COLS = 512;
@@ -294,7 +301,7 @@ __device__ __forceinline__ void dropout_keep_keyrow_64(uint32_t (&mask)[2], int 
 //   dV += (P*Z)^T dO * s,   dS = P * (Z * s * dP - D),   s = 256 / t.
 template <int D, bool WIN, bool DROP = false>
 __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
-  using C = BwdCfg<D>;
+  using C = BwdCfg<D, DROP>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {  // the layout needs 1024-byte aligned swizzle atoms
@@ -319,6 +326,10 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
   const uint32_t bar_p_read = bar0 + 8u * 24;    // the dS warps hold this tile's P^T
   const uint32_t bar_do_empty = bar0 + 8u * 25;
   const uint32_t bar_ds_free = bar0 + 8u * 26;   // d = 64: the tile's dQ and dK have read the dS tile
+  // dropout keep bits of query tile gi in buffer gi & 1: written by the mask
+  // warps, read by every P^T thread
+  auto bar_mask_full = [&](int b) { return bar0 + 8u * (27 + b); };
+  auto bar_mask_empty = [&](int b) { return bar0 + 8u * (29 + b); };
   // Q/dO stage of global iteration g and the parity of its use of that stage.
   auto stg = [&](int g) { return g % C::NQ; };
   auto stg_par = [&](int g) { return (uint32_t)((g / C::NQ) & 1); };
@@ -359,6 +370,12 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
     mbar_init(bar_do_empty, 1);
     mbar_init(bar_p_read, 256);
     mbar_init(bar_ds_free, 1);
+    if (C::MASKW) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(bar_mask_full(b), 64);
+        mbar_init(bar_mask_empty(b), 256);
+      }
+    }
     fence_barrier_init();
   }
   if (warp == C::MMA_WARP) {
@@ -426,6 +443,52 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         for (int g = max(0, gi - C::NQ); g <= gi; ++g)
           mbar_wait_drain(bar_qdo_full(stg(g)), stg_par(g), p.wait_limit_ns);
         if (n_do > 0) mbar_wait_drain(bar_do_full, (n_do - 1) & 1, p.wait_limit_ns);
+      }
+    }
+  } else if (C::MASKW && warp >= 22) {
+    // ------------------------------------------------------------ dropout mask
+    // Thread mt makes the keep bits of keys 4 (mt >> 1) .. + 3 of the tile for
+    // query half mt & 1 of every query tile: the 16 Philox blocks of those
+    // keys and 64 queries (the layout the P^T warps' own generator uses:
+    // counter (query / 4, key / 4, bh, offset), word = query, byte = key),
+    // each key's bits gathered into two 32-query words.
+    const int mt = threadIdx.x - 704;
+    const int cl = mt >> 1, half = mt & 1;
+    const uint32_t tt = p.drop_t * 0x01010101u;
+    uint2* mbuf = reinterpret_cast<uint2*>(smem + C::OFF_MASK);
+    bool ok = true;
+    int gi = 0;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const BwdItem I = bwd_item(p, item);
+      const uint32_t cg = (uint32_t)(I.j0 >> 2) + (uint32_t)cl;
+      for (int it = 0; it < I.n_it && ok; ++it, ++gi) {
+        const int mb = gi & 1;
+        if (gi >= 2) ok = mbar_wait(bar_mask_empty(mb), ((gi >> 1) - 1) & 1, wc);
+        if (!ok) break;
+        const uint32_t bh = (uint32_t)(I.b * p.Hq + I.hkv * G + it / I.nq);
+        const uint32_t a0 = (uint32_t)((I.qt_begin + it % I.nq) * 128 + 64 * half) >> 2;
+        uint32_t kw[4][2];  // [key of the group][32-query word]
+#pragma unroll
+        for (int w2 = 0; w2 < 2; ++w2) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) kw[r][w2] = 0u;
+          // rolled: unrolled, the blocks' states would not fit 80 registers
+#pragma unroll 1
+          for (int al = 0; al < 8; ++al) {
+            const uint4 wv = philox4x32_10(make_uint4(a0 + 8 * w2 + al, cg, bh, p.drop_offset), p.seed_lo, p.seed_hi);
+            // 4 x 4 byte transpose: x[r] = byte r (key 4 cg + r) of words 0..3
+            // (queries)
+            const uint32_t lo01 = __byte_perm(wv.x, wv.y, 0x5140), hi01 = __byte_perm(wv.x, wv.y, 0x7362);
+            const uint32_t lo23 = __byte_perm(wv.z, wv.w, 0x5140), hi23 = __byte_perm(wv.z, wv.w, 0x7362);
+            const uint32_t x[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
+                                   __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) kw[r][w2] |= gather_msb4(bytes_below(x[r], tt)) << (4 * al);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) mbuf[(mb * 128 + 4 * cl + r) * 2 + half] = make_uint2(kw[r][0], kw[r][1]);
+        mbar_arrive(bar_mask_full(mb));
       }
     }
   } else if (warp == C::MMA_WARP) {
@@ -595,9 +658,19 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         // dropout: this key's keep bits for the warp's 64 queries, made while
         // the tensor core computes S^T
         uint32_t keep[2] = {0u, 0u};
-        if constexpr (DROP)
+        if constexpr (C::MASKW) {
+          // this key's keep bits for the warp's 64 queries, from the mask warps
+          const int mb = gi & 1;
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_mask_full(mb), (gi >> 1) & 1, wc));
+          if (!ok) break;
+          const uint2 kv = reinterpret_cast<const uint2*>(smem + C::OFF_MASK)[(mb * 128 + j) * 2 + half];
+          keep[0] = kv.x;
+          keep[1] = kv.y;
+          mbar_arrive(bar_mask_empty(mb));
+        } else if constexpr (DROP) {
           dropout_keep_keyrow_64(keep, key, q0 + 64 * half, (uint32_t)(I.b * p.Hq + I.hkv * G + it / I.nq),
                                  p.drop_offset, p.seed_lo, p.seed_hi, p.drop_t);
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo_full(s), stg_par(gi), wc));
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(buf), (gi / C::NSBUF) & 1, wc));
         if (!ok) break;
@@ -883,7 +956,7 @@ static int bwd_setup() {
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false, true>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false, true>)};
   const int bytes[6] = {BwdCfg<64>::SMEM_BYTES, BwdCfg<64>::SMEM_BYTES, BwdCfg<128>::SMEM_BYTES,
-                        BwdCfg<128>::SMEM_BYTES, BwdCfg<64>::SMEM_BYTES, BwdCfg<128>::SMEM_BYTES};
+                        BwdCfg<128>::SMEM_BYTES, BwdCfg<64, true>::SMEM_BYTES, BwdCfg<128, true>::SMEM_BYTES};
   for (int i = 0; i < 6; ++i)
     if (cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes[i]) != cudaSuccess)
       return FA_ERR_CUDA;

@@ -101,3 +101,29 @@ def test_dropout_backward_zero_rate_is_the_plain_backward():
         # dQ adds fp32 contributions in an unspecified order; dK and dV are exact
         assert torch.allclose(a.float(), b.float(), rtol=1e-2, atol=1e-3)
     assert torch.equal(g0[1], g1[1]) and torch.equal(g0[2], g1[2])
+
+
+def test_dropout_persistent_items_d64():
+    """d = 64 runs persistently (one CTA per SM walks several items), and its
+    keep bits come from dedicated warps through double-buffered shared
+    memory that carries over from one item to the next.  With 256 forward
+    and 512 backward items on 148 SMs, the heads checked here are second or
+    later items of their CTAs; each is compared with the oracle's per-head
+    dropout forward and backward (same Philox mask, bh = b * Hq + h)."""
+    B, H, T, d, p = 4, 16, 1024, 64, 0.1
+    w = WORKLOADS[2].with_(B=B, Hq=H, Hkv=H, d=d, causal=False)
+    inp = prefill_inputs(w, seed=1234, Tq=T, Tk=T)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "do"))
+    seed, offset = 0x1234_5678_9ABC, 7
+    o, lse = fa.forward_dropout(q, k, v, p, seed, offset, scale=w.scale, causal=False)
+    dq, dk, dv = fa.backward_dropout(q, k, v, o, lse, do, p, seed, offset, scale=w.scale, causal=False)
+    assert fa.check() == 0
+    back = dr.keep_threshold(p) / 256.0
+    for b, h in ((1, 4), (2, 8), (3, 15)):
+        qh, kh, vh, doh = (to_f64(inp[n][b, :, h]) for n in ("q", "k", "v", "do"))
+        O, LSE = dr.head_forward_dropout(qh, kh, vh, w.scale, False, p, seed, offset, b * H + h)
+        assert_o_close(to_f64(o[b, :, h].cpu()) * back, O * back, f"O[{b},{h}]")
+        assert_lse_close(lse[b, h].cpu().numpy(), LSE, f"LSE[{b},{h}]")
+        rq, rk, rv = dr.head_backward_dropout(qh, kh, vh, doh, w.scale, False, p, seed, offset, b * H + h)
+        for name, x, r in (("dQ", dq[b, :, h], rq), ("dK", dk[b, :, h], rk), ("dV", dv[b, :, h], rv)):
+            assert_grad_close(to_f64(x.cpu()), r, f"{name}[{b},{h}]")

@@ -92,6 +92,25 @@ def test_window_long_sequence_sampled_rows():
         assert_lse_close(lse[0, h, rows].numpy(), LSE)
 
 
+def test_window_persistent_items_sampled_rows():
+    """Windowed forwards run persistently (one CTA per SM walks several
+    items): with 16 heads of T = 8192 there are 512 items on 148 SMs, and
+    heads 7 and 15 are second or later items of their CTAs.  Sampled rows
+    against the oracle."""
+    w = WORKLOADS[3].with_(B=1, Hq=16, Hkv=16)
+    W = 1024
+    inp = prefill_inputs(w, device="cuda")
+    o, lse = fa.forward(inp["q"], inp["k"], inp["v"], scale=w.scale, window=W)
+    assert fa.check() == 0
+    o, lse = o.cpu(), lse.cpu()
+    rows = np.array([0, 255, 256, 1023, 1024, 4097, 8191])
+    for h in (7, 15):
+        q64, k64, v64 = (to_f64(inp[n][0, :, h].cpu()) for n in ("q", "k", "v"))
+        O, LSE = oracle.head_forward(q64, k64, v64, w.scale, True, rows=rows, window=W)
+        assert_o_close(to_f64(o[0, rows, h]), O)
+        assert_lse_close(lse[0, h, rows].numpy(), LSE)
+
+
 @pytest.mark.parametrize("Hq,Hkv,d,chunk,W,seqlens", [
     (8, 2, 128, 256, 300, [1, 255, 256, 257, 1000]),   # window inside, across and beyond chunks
     (4, 4, 64, 256, 1, [1, 64, 65, 777]),              # the last key only

@@ -99,3 +99,17 @@ def test_fp8_forward_gqa_long_context_sampled_rows():
     rows = [0, 1, 2, 127, 128, 255, 4096, 16383, 16384, 32766, 32767]
     for h in (0, 3, 28, 31):
         _check_head(o, lse, inp, 0, h, w.Hq // w.Hkv, w.scale, True, rows=rows)
+
+
+def test_fp8_forward_persistent_items_sampled_rows():
+    """Non-causal E4M3 launches are persistent (one CTA per SM walks several
+    items): B 2, Hq 32, Hkv 8, T 4096 gives 1024 items on 148 SMs, and the
+    heads checked are later items of their CTAs.  Sampled rows."""
+    w = WORKLOADS[3].with_(B=2, Hq=32, Hkv=8, causal=False)
+    inp = prefill_inputs_e4m3(w, seed=29, Tq=4096, Tk=4096, device="cuda")
+    o, lse = fa.forward_fp8(inp["q"], inp["k"], inp["v"], inp["q_descale"], inp["k_descale"], inp["v_descale"],
+                            scale=w.scale, causal=False)
+    assert fa.check() == 0
+    rows = [0, 127, 128, 2047, 2048, 4095]
+    for b, h in ((0, 15), (1, 31)):
+        _check_head(o, lse, inp, b, h, w.Hq // w.Hkv, w.scale, False, rows=rows)

@@ -201,8 +201,8 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_MASK + MASK_BYTES;
   // kv_full[2], kv_empty[2], qdo_full[3], qdo_empty[3], s_full[2], p_full[2],
   // dp_full, ds_full, dq_full[2], dq_free[2], dkdv_done, mma_done, dp_free,
-  // do_full, p_read, do_empty, ds_free (, mask_full[2], mask_empty[2])
-  static constexpr int NBAR = 27 + (MASKW ? 4 : 0);
+  // do_full, p_read, do_empty (, mask_full[2], mask_empty[2])
+  static constexpr int NBAR = 26 + (MASKW ? 4 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   // warps 0-7 P^T (two per TMEM lane quarter, one per half of the query
@@ -325,11 +325,10 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
   const uint32_t bar_do_full = bar0 + 8u * 23;   // single dO buffer (d = 128)
   const uint32_t bar_p_read = bar0 + 8u * 24;    // the dS warps hold this tile's P^T
   const uint32_t bar_do_empty = bar0 + 8u * 25;
-  const uint32_t bar_ds_free = bar0 + 8u * 26;   // d = 64: the tile's dQ and dK have read the dS tile
   // dropout keep bits of query tile gi in buffer gi & 1: written by the mask
   // warps, read by every P^T thread
-  auto bar_mask_full = [&](int b) { return bar0 + 8u * (27 + b); };
-  auto bar_mask_empty = [&](int b) { return bar0 + 8u * (29 + b); };
+  auto bar_mask_full = [&](int b) { return bar0 + 8u * (26 + b); };
+  auto bar_mask_empty = [&](int b) { return bar0 + 8u * (28 + b); };
   // Q/dO stage of global iteration g and the parity of its use of that stage.
   auto stg = [&](int g) { return g % C::NQ; };
   auto stg_par = [&](int g) { return (uint32_t)((g / C::NQ) & 1); };
@@ -369,7 +368,6 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
     mbar_init(bar_do_full, 1);
     mbar_init(bar_do_empty, 1);
     mbar_init(bar_p_read, 256);
-    mbar_init(bar_ds_free, 1);
     if (C::MASKW) {
       for (int b = 0; b < 2; ++b) {
         mbar_init(bar_mask_full(b), 64);
@@ -598,9 +596,10 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           // columns, which the dS warps have read (the S^T buffer already
           // holds the next S^T).  At d = 64 dQ goes first, so that its
           // read-out, which the next-but-one S^T waits for, starts one
-          // product earlier (measured 6% faster), and a separate commit
-          // after dK frees the dS tile; at d = 128 dK first measured faster,
-          // and dQ's completion frees the tile.
+          // product earlier (measured 6% faster), and dK's commit, which
+          // frees the Q stage, also frees the dS tile (the dS warps wait on
+          // the stage's barrier); at d = 128 dK first measured faster, and
+          // dQ's completion frees the tile.
           const uint32_t tDQ = C::NSBUF == 1 ? tDP : tS(buf);
           if constexpr (D == 64) {
 #pragma unroll
@@ -610,7 +609,6 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             for (int k = 0; k < 8; ++k)
               mma_ss(tDK, kdesc(aDS, k), mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
             mma_commit(bar_qdo_empty(stg(gi)));
-            mma_commit(bar_ds_free);
           } else {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
@@ -845,7 +843,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             // dK and dQ MMAs until they complete (this tile's dP^T can
             // complete before them).
             ok = __all_sync(0xffffffffu,
-                            D == 64 ? mbar_wait(bar_ds_free, (gi - 1) & 1, wc)
+                            D == 64 ? mbar_wait(bar_qdo_empty(stg(gi - 1)), stg_par(gi - 1), wc)
                                     : mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
             if (!ok) break;
           }

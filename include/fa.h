@@ -175,6 +175,26 @@ int fa_backward_window(const void* q, const void* k, const void* v, const void* 
                        void* stream);
 
 /*
+ * fa_backward_deterministic -- the gradients of fa_backward (causal = 0 or 1,
+ * window = 0) or of fa_backward_window (causal = 1, window >= 1), with dQ
+ * the same bit for bit from run to run.  fa_backward adds every KV tile's
+ * share of dQ into an fp32 accumulator with bulk reduce-adds, whose order
+ * varies between runs; here the dK/dV pass leaves dQ out and a second pass,
+ * one work item per (128-query tile, head, batch), recomputes S and dP for
+ * the tile's KV tiles, keeps dQ in tensor memory and writes it once
+ * ("FlashAttention", follow-up on recomputing instead of storing P).  dK and
+ * dV are those of fa_backward, bit for bit.  It costs more time: the second
+ * pass recomputes the two products S and dP.  Arguments, workspace and
+ * errors as fa_backward; window < 0, or window > 0 without causal = 1, is
+ * FA_ERR_INVALID_ARG.  bf16, d = 64 or 128, no dropout.
+ */
+int fa_backward_deterministic(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                              void* ws, size_t ws_bytes,
+                              int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale,
+                              int causal, int window, void* stream);
+
+/*
  * The three steps fa_backward runs, in this order on one stream, exposed so
  * that a caller can schedule or time them separately.  They share the
  * workspace of fa_backward_workspace_bytes() and its layout; arguments mean

@@ -39,6 +39,8 @@ SIGNATURES = {
     "fa_backward_workspace_bytes": (_c_size, [_c_int] * 6),
     "fa_backward": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
     "fa_backward_window": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _vp]),
+    "fa_backward_deterministic": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _c_int,
+                                                                                      _vp]),
     "fa_backward_dropout": (_c_int, [_vp] * 9 + [_vp, _c_size] + [_c_int] * 6 + [_c_float, _c_int, _c_float,
                                                                              ctypes.c_ulonglong, ctypes.c_uint, _vp]),
     "fa_backward_dkdv_dropout": (_c_int, [_vp] * 7 + [_c_size] + [_c_int] * 6 + [_c_float, _c_int, _c_float,
@@ -198,9 +200,11 @@ def backward_workspace_bytes(B, Hq, Hkv, Tq, Tk, d) -> int:
 
 
 def backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None, dq=None, dk=None, dv=None,
-             window=None):
+             window=None, deterministic=False):
     """dQ, dK, dV for L = sum(dO * O).  `workspace` (uint8 CUDA tensor) is
-    allocated here when not given; ``window`` as in forward()."""
+    allocated here when not given; ``window`` as in forward().
+    ``deterministic``: fa_backward_deterministic (dQ the same bit for bit from
+    run to run, at the cost of a second pass)."""
     lib = load_library()
     B, Tq, Hq, d = q.shape
     Tk, Hkv = k.shape[1], k.shape[2]
@@ -218,7 +222,11 @@ def backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None, dq=N
     dv = torch.empty_like(v) if dv is None else dv
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
             _ptr(workspace), workspace.numel(), B, Hq, Hkv, Tq, Tk, d, float(scale))
-    if window is None:
+    if deterministic:
+        win = 0 if window is None else int(window)
+        st = lib.fa_backward_deterministic(*args, int(bool(causal) or win > 0), win, _stream_ptr(dev))
+        _raise("fa_backward_deterministic", st)
+    elif window is None:
         st = lib.fa_backward(*args, int(bool(causal)), _stream_ptr(dev))
         _raise("fa_backward", st)
     else:

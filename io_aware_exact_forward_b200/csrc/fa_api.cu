@@ -15,6 +15,7 @@
 #include "fa_ptx.cuh"
 #include "fa_fwd.cuh"
 #include "fa_bwd.cuh"
+#include "fa_bwd_dq.cuh"
 #include "fa_decode.cuh"
 
 namespace fa {
@@ -143,6 +144,7 @@ static int device_setup_impl() {
   if (!st) st = fwd_setup_one<64, false, true>();
   if (!st) st = fwd_setup_one<128, false, true>();
   if (!st) st = bwd_setup();
+  if (!st) st = bwd_dq_setup();
   if (!st) st = decode_setup();
   return st;
 }
@@ -360,8 +362,10 @@ static int check_ptrs(std::initializer_list<const void*> ptrs) {
   return FA_OK;
 }
 
-int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void* ws, size_t ws_bytes,
-                           int B, int Hq, int Hkv, int Tq, int Tk, int d, void* stream) {
+// zero_acc = false leaves the fp32 dQ accumulator alone (a backward whose dQ
+// pass writes dq directly does not read it).
+static int preprocess_impl(const void* o, const float* lse, const void* dO, void* ws, size_t ws_bytes, int B,
+                           int Hq, int Hkv, int Tq, int Tk, int d, void* stream, bool zero_acc) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, 1.f, 0);
   if (st) return st;
   if (B == 0 || Tq == 0) return FA_OK;
@@ -375,21 +379,30 @@ int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const __nv_bfloat16* o16 = reinterpret_cast<const __nv_bfloat16*>(o);
   const __nv_bfloat16* do16 = reinterpret_cast<const __nv_bfloat16*>(dO);
+  float* acc = zero_acc ? w.dq_acc : nullptr;
   if (d == 64)
-    fa_bwd_preprocess_kernel<64><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, w.dq_acc, B, Hq, Tq, Tp);
+    fa_bwd_preprocess_kernel<64><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, acc, B, Hq, Tq, Tp);
   else
-    fa_bwd_preprocess_kernel<128><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, w.dq_acc, B, Hq, Tq, Tp);
+    fa_bwd_preprocess_kernel<128><<<blocks, 256, 0, s>>>(o16, do16, lse, w.Dv, w.lse2, acc, B, Hq, Tq, Tp);
   return launch_status();
+}
+
+int fa_backward_preprocess(const void* o, const float* lse, const void* dO, void* ws, size_t ws_bytes,
+                           int B, int Hq, int Hkv, int Tq, int Tk, int d, void* stream) {
+  return preprocess_impl(o, lse, dO, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream, true);
 }
 
 }  // extern "C"
 
 // drop_t in 1..255: dropout on P with that keep threshold and Philox key
 // (seed_lo, seed_hi), counter word drop_offset (the forward's mask).
+// det: dQ from the separate, deterministic pass (fa_bwd_dq.cuh) after the
+// dK/dV kernel built without dQ, into the fp32 accumulator or, when dq_out
+// is given, as bf16 straight into dq_out (no dropout).
 static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* ws,
                      size_t ws_bytes, int B, int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal,
                      int window, void* stream, uint32_t drop_t = 256, uint32_t seed_lo = 0, uint32_t seed_hi = 0,
-                     uint32_t drop_offset = 0) {
+                     uint32_t drop_offset = 0, bool det = false, void* dq_out = nullptr) {
   const bool drop = drop_t < 256;
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
@@ -437,23 +450,65 @@ static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO
   const bool persistent = d == 64 && !causal;
   dim3 grid(persistent ? std::min(p.n_items, nsm) : p.n_items);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (drop && window > 0) return FA_ERR_UNSUPPORTED;
+  if (drop && (window > 0 || det)) return FA_ERR_UNSUPPORTED;
   if (drop) {
     if (d == 64)
       fa_bwd_dkdv_kernel<64, false, true><<<grid, BwdCfg<64, true>::THREADS, BwdCfg<64, true>::SMEM_BYTES, s>>>(p);
     else
       fa_bwd_dkdv_kernel<128, false, true><<<grid, BwdCfg<128, true>::THREADS, BwdCfg<128, true>::SMEM_BYTES, s>>>(p);
-  } else if (d == 64) {
-    if (window > 0)
+    return launch_status();
+  }
+  if (!det) {
+    if (d == 64 && window > 0)
       fa_bwd_dkdv_kernel<64, true><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
-    else
+    else if (d == 64)
       fa_bwd_dkdv_kernel<64, false><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
-  } else {
-    if (window > 0)
+    else if (window > 0)
       fa_bwd_dkdv_kernel<128, true><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
     else
       fa_bwd_dkdv_kernel<128, false><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+    return launch_status();
   }
+  // deterministic: dK/dV without dQ, then the dQ pass
+  if (d == 64 && window > 0)
+    fa_bwd_dkdv_kernel<64, true, false, false><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+  else if (d == 64)
+    fa_bwd_dkdv_kernel<64, false, false, false><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+  else if (window > 0)
+    fa_bwd_dkdv_kernel<128, true, false, false><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+  else
+    fa_bwd_dkdv_kernel<128, false, false, false><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+  if ((st = launch_status())) return st;
+  if (Tq == 0) return FA_OK;
+  DqParams qp;
+  memset(&qp, 0, sizeof(qp));
+  qp.tm_q = p.tm_q;
+  qp.tm_do = p.tm_do;
+  qp.tm_k = p.tm_k;
+  qp.tm_v = p.tm_v;
+  qp.lse2 = w.lse2;
+  qp.Dv = w.Dv;
+  qp.dq_acc = w.dq_acc;
+  qp.dq = reinterpret_cast<__nv_bfloat16*>(dq_out);
+  qp.B = B; qp.Hq = Hq; qp.Hkv = Hkv; qp.Tq = Tq; qp.Tk = Tk; qp.causal = causal;
+  qp.window = window;
+  qp.Tq_pad = p.Tq_pad;
+  qp.scale = scale;
+  qp.scale_log2 = p.scale_log2;
+  qp.n_qt = (Tq + 127) / 128;
+  const long long n_items = (long long)B * Hq * qp.n_qt;
+  if (n_items > 0x7FFFFFFFll) return FA_ERR_INVALID_ARG;
+  qp.n_items = (int)n_items;
+  qp.wait_limit_ns = kWaitLimitNs;
+  const unsigned nblk = (unsigned)qp.n_items;
+  if (d == 64 && window > 0)
+    fa_bwd_dq_kernel<64, true><<<nblk, DqCfg<64>::THREADS, DqCfg<64>::SMEM_BYTES, s>>>(qp);
+  else if (d == 64)
+    fa_bwd_dq_kernel<64, false><<<nblk, DqCfg<64>::THREADS, DqCfg<64>::SMEM_BYTES, s>>>(qp);
+  else if (window > 0)
+    fa_bwd_dq_kernel<128, true><<<nblk, DqCfg<128>::THREADS, DqCfg<128>::SMEM_BYTES, s>>>(qp);
+  else
+    fa_bwd_dq_kernel<128, false><<<nblk, DqCfg<128>::THREADS, DqCfg<128>::SMEM_BYTES, s>>>(qp);
   return launch_status();
 }
 
@@ -503,7 +558,7 @@ static int backward_impl(const void* q, const void* k, const void* v, const void
                          const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B, int Hq,
                          int Hkv, int Tq, int Tk, int d, float scale, int causal, int window, void* stream,
                          uint32_t drop_t = 256, uint32_t seed_lo = 0, uint32_t seed_hi = 0,
-                         uint32_t drop_offset = 0) {
+                         uint32_t drop_offset = 0, bool det = false) {
   int st = check_prefill(B, Hq, Hkv, Tq, Tk, d, scale, causal);
   if (st) return st;
   if (window < 0 || window > (1 << 30)) return FA_ERR_INVALID_ARG;
@@ -511,10 +566,14 @@ static int backward_impl(const void* q, const void* k, const void* v, const void
   if (Tq > 0 && (st = check_ptrs({q, o, lse, dO, dq}))) return st;
   if (Tk > 0 && (st = check_ptrs({k, v, dk, dv}))) return st;
   if ((st = check_ws(ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d))) return st;
-  if ((st = fa_backward_preprocess(o, lse, dO, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream))) return st;
+  // deterministic: the dQ pass writes dq itself (when there are keys; with
+  // none, dq is the zeroed accumulator converted)
+  const bool direct = det && Tq > 0 && Tk > 0;
+  if ((st = preprocess_impl(o, lse, dO, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream, !direct))) return st;
   if ((st = dkdv_impl(q, k, v, dO, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, window, stream,
-                      drop_t, seed_lo, seed_hi, drop_offset)))
+                      drop_t, seed_lo, seed_hi, drop_offset, det, direct ? dq : nullptr)))
     return st;
+  if (direct) return FA_OK;
   return fa_backward_dq_finalize(dq, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, stream);
 }
 
@@ -543,6 +602,15 @@ int fa_backward_window(const void* q, const void* k, const void* v, const void* 
   if (window < 1) return FA_ERR_INVALID_ARG;
   return backward_impl(q, k, v, o, lse, dO, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, 1, window,
                        stream);
+}
+
+int fa_backward_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dO, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B,
+                              int Hq, int Hkv, int Tq, int Tk, int d, float scale, int causal, int window,
+                              void* stream) {
+  if (window < 0 || (window > 0 && causal != 1)) return FA_ERR_INVALID_ARG;
+  return backward_impl(q, k, v, o, lse, dO, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, Tq, Tk, d, scale, causal, window,
+                       stream, 256, 0, 0, 0, true);
 }
 
 static size_t decode_nchunk(int Tk_max, int chunk) { return ((size_t)Tk_max + chunk - 1) / chunk; }

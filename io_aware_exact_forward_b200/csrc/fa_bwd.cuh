@@ -8,7 +8,7 @@
 // Three kernels:
 //   preprocess   D_i = sum_c dO_ic O_ic (fp32), LSE in log2 units (+inf for a
 //                row that saw no key, so that its P is exactly 0), dQ
-//                accumulator zeroed.                          (memory-bound)
+//                accumulator zeroed (unless dq_acc is null). (memory-bound)
 //   dkdv         one work item per (128-key tile, KV head, batch).  K and V
 //                stay in shared memory; the item walks the query tiles of
 //                every query head of its GQA group.  Per tile:
@@ -76,9 +76,11 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(
       dot = fmaf(x.x, y.x, dot);
       dot = fmaf(x.y, y.y, dot);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + sub * 8);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (dq_acc) {
+      float4* z = reinterpret_cast<float4*>(dq_acc + row * D + sub * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int off = LPR / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
@@ -293,13 +295,15 @@ __device__ __forceinline__ void dropout_keep_keyrow_64(uint32_t (&mask)[2], int 
 }
 
 // WIN: sliding-window masking compiled in (a separate instantiation, so
-// that the plain path keeps its registers).  DROP: dropout on P, with the
+// that the plain path keeps its registers).  DQ = false: no dQ product,
+// read-out or reduce-adds (warps 16-19 idle); dQ then comes from the
+// separate, deterministic pass of fa_bwd_dq.cuh.  DROP: dropout on P, with the
 // keep mask of the forward regenerated per key row; the P^T warps write the
 // dropped P^T (the dV operand) and the undropped P^T side by side, 8 columns
 // each per 16-query chunk, and the dS warps read the keep bits off the
 // dropped copy's zeros:
 //   dV += (P*Z)^T dO * s,   dS = P * (Z * s * dP - D),   s = 256 / t.
-template <int D, bool WIN, bool DROP = false>
+template <int D, bool WIN, bool DROP = false, bool DQ = true>
 __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D, DROP>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -358,7 +362,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
       mbar_init(bar_s_full(s), 1);
       mbar_init(bar_p_full(s), 256);
       mbar_init(bar_dq_full(s), 1);
-      mbar_init(bar_dq_free(s), 128);
+      mbar_init(bar_dq_free(s), DQ ? 128 : 256);
     }
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_dp_free, 256);
@@ -550,7 +554,11 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           };
           if (C::NSBUF == 2 && has_next) {
             // S^T of the next iteration into the other buffer, which dQ of
-            // the previous iteration used.
+            // the previous iteration used.  Without dQ the buffer's dq_free
+            // barrier is arrived on by the dS warps once they hold that
+            // iteration's P^T (its dV, issued earlier, reads P^T ahead of
+            // the new S^T in the tensor pipe's order); a barrier per buffer,
+            // so that the awaited phase is never two behind.
             ok = wait_next_operands();
             if (ok && gi >= 1) ok = mbar_wait(bar_dq_free((gi + 1) & 1), ((gi - 1) >> 1) & 1, wc);
             if (!ok) break;
@@ -602,9 +610,11 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
           // dQ's completion frees the tile.
           const uint32_t tDQ = C::NSBUF == 1 ? tDP : tS(buf);
           if constexpr (D == 64) {
+            if constexpr (DQ) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
-            mma_commit(bar_dq_full(buf));
+              for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
+              mma_commit(bar_dq_full(buf));
+            }
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               mma_ss(tDK, kdesc(aDS, k), mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
@@ -614,17 +624,20 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             for (int k = 0; k < 8; ++k)
               mma_ss(tDK, kdesc(aDS, k), mndesc(aQ(gi), k), C::IDESC_TS, it > 0 || k > 0);
             mma_commit(bar_qdo_empty(stg(gi)));
+            if constexpr (DQ) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
-            mma_commit(bar_dq_full(buf));
+              for (int k = 0; k < 8; ++k) mma_ss(tDQ, mndesc(aDS, k), mndesc(aK(kvb), k), C::IDESC_DQ, k > 0);
+              mma_commit(bar_dq_full(buf));
+            }
           }
           if (last) {
             mma_commit(bar_kv_empty(kvb));
             mma_commit(bar_dkdv_done);
           }
           if (C::NSBUF == 1 && has_next) {
-            // The next dP^T reuses the dQ columns: after the dQ read-out.
-            ok = mbar_wait(bar_dq_free(0), gi & 1, wc);
+            // The next dP^T reuses the dQ columns: after the dQ read-out
+            // (without dQ, once the dS warps have read this dP^T).
+            ok = DQ ? mbar_wait(bar_dq_free(0), gi & 1, wc) : mbar_wait(bar_dp_free, gi & 1, wc);
             if (ok) ok = wait_do(gi + 1);
             if (!ok) break;
             tc_fence_after();
@@ -805,6 +818,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar_p_read);
+        if constexpr (!DQ && C::NSBUF == 2) mbar_arrive(bar_dq_free(buf));
         ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, gi & 1, wc));
         if (!ok) break;
         tc_fence_after();
@@ -843,7 +857,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
             // dK and dQ MMAs until they complete (this tile's dP^T can
             // complete before them).
             ok = __all_sync(0xffffffffu,
-                            D == 64 ? mbar_wait(bar_qdo_empty(stg(gi - 1)), stg_par(gi - 1), wc)
+                            (D == 64 || !DQ) ? mbar_wait(bar_qdo_empty(stg(gi - 1)), stg_par(gi - 1), wc)
                                     : mbar_wait(bar_dq_full((gi - 1) % C::NSBUF), ((gi - 1) / C::NSBUF) & 1, wc));
             if (!ok) break;
           }
@@ -862,7 +876,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         mbar_arrive(bar_ds_full);
       }
     }
-  } else if (warp < 20) {
+  } else if (DQ && warp < 20) {
     // ------------------------------------------------------------ dQ (WG-C)
     const int r = threadIdx.x - 512;         // query row in the tile == TMEM lane
     const int lead = 512;                    // thread that issues the bulk reduces
@@ -947,15 +961,21 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
 }
 
 static int bwd_setup() {
-  const void* kernels[6] = {reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false>),
+  const void* kernels[10] = {reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, true>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, true>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false, true>),
-                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false, true>)};
-  const int bytes[6] = {BwdCfg<64>::SMEM_BYTES, BwdCfg<64>::SMEM_BYTES, BwdCfg<128>::SMEM_BYTES,
-                        BwdCfg<128>::SMEM_BYTES, BwdCfg<64, true>::SMEM_BYTES, BwdCfg<128, true>::SMEM_BYTES};
-  for (int i = 0; i < 6; ++i)
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false, true>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, false, false, false>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, true, false, false>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false, false, false>),
+                            reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, true, false, false>)};
+  const int bytes[10] = {BwdCfg<64>::SMEM_BYTES,       BwdCfg<64>::SMEM_BYTES,       BwdCfg<128>::SMEM_BYTES,
+                         BwdCfg<128>::SMEM_BYTES,      BwdCfg<64, true>::SMEM_BYTES, BwdCfg<128, true>::SMEM_BYTES,
+                         BwdCfg<64>::SMEM_BYTES,       BwdCfg<64>::SMEM_BYTES,       BwdCfg<128>::SMEM_BYTES,
+                         BwdCfg<128>::SMEM_BYTES};
+  for (int i = 0; i < 10; ++i)
     if (cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes[i]) != cudaSuccess)
       return FA_ERR_CUDA;
   return FA_OK;

@@ -267,6 +267,36 @@ def cpu_baseline(w, inp_cpu, budget_s):
                       f"({dt:.1f} s; same algorithmic FLOP count as the GPU metric)"}
 
 
+def cpu_sdpa_fp32(w, inp_cpu, budget_s):
+    """torch's own CPU scaled_dot_product_attention in fp32, forward and
+    backward through autograd, one batch entry (all its heads) at a time
+    until the budget is spent: a second, less deliberately slow CPU figure
+    beside the float64 oracle (the same algorithmic FLOP count)."""
+    import torch
+    import torch.nn.functional as F
+    G = w.Hq // w.Hkv
+    pairs = w.T * (w.T + 1) // 2 if w.causal else w.T * w.T
+    fl_one = 14 * w.Hq * w.d * pairs
+    done, dt, warm = 0, 0.0, False
+    for b in [0] + list(range(w.B)):  # the first pass (batch entry 0) warms up, untimed
+        q = inp_cpu["q"][b].float().transpose(0, 1).contiguous().requires_grad_()        # [Hq, T, d]
+        k = inp_cpu["k"][b].float().transpose(0, 1).repeat_interleave(G, 0).contiguous().requires_grad_()
+        v = inp_cpu["v"][b].float().transpose(0, 1).repeat_interleave(G, 0).contiguous().requires_grad_()
+        do = inp_cpu["do"][b].float().transpose(0, 1).contiguous()
+        t0 = time.perf_counter()
+        o = F.scaled_dot_product_attention(q, k, v, is_causal=w.causal, scale=w.scale)
+        o.backward(do)
+        if warm:
+            dt += time.perf_counter() - t0
+            done += 1
+            if dt >= budget_s:
+                break
+        warm = True
+    return {"value": fl_one * done / dt / 1e12, "unit": "TFLOP/s", "cores": torch.get_num_threads(),
+            "kind": "torch CPU scaled_dot_product_attention, fp32, forward + backward (autograd)",
+            "sample": f"{done} of {w.B} batch entries (all {w.Hq} heads each) of {w.name} ({dt:.1f} s)"}
+
+
 # ---------------------------------------------------------------------------
 # reference arm
 # ---------------------------------------------------------------------------
@@ -730,6 +760,9 @@ def run_fa(args, w, rank, world, dist):
         inp_cpu = {"q": q.cpu(), "k": k.cpu(), "v": v.cpu(), "do": do.cpu()}
         cpu = cpu_baseline(w, inp_cpu, args.cpu_seconds)
         cpu["tokens_per_s"] = cpu["value"] * 1e12 / ((f_fwd + f_bwd) / prefill_tokens(w))
+        sdpa = cpu_sdpa_fp32(w, inp_cpu, min(args.cpu_seconds, 10.0))
+        sdpa["tokens_per_s"] = sdpa["value"] * 1e12 / ((f_fwd + f_bwd) / prefill_tokens(w))
+        cpu["second_baseline"] = sdpa
 
     extras = None
     if args.workload == 2 and not w.window and args.batch is None and not args.no_extra:

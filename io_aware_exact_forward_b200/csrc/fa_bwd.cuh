@@ -375,7 +375,7 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
     if (C::MASKW) {
       for (int b = 0; b < 2; ++b) {
         mbar_init(bar_mask_full(b), 64);
-        mbar_init(bar_mask_empty(b), 256);
+        mbar_init(bar_mask_empty(b), 512);  // the P^T and the dS warps read each buffer
       }
     }
     fence_barrier_init();
@@ -797,7 +797,19 @@ __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdPa
         // that the S^T buffer can take the next S^T.
         uint32_t pp[32];
         uint32_t keep[2] = {0u, 0u};
-        if constexpr (DROP) {
+        if constexpr (C::MASKW) {
+          // undropped P^T, and this key's keep bits from the mask warps'
+          // buffer (as the P^T warps read them)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld8(tP + 16 * c + 8, pp + 8 * c);
+          const int mb = gi & 1;
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_mask_full(mb), (gi >> 1) & 1, wc));
+          if (!ok) break;
+          const uint2 kv = reinterpret_cast<const uint2*>(smem + C::OFF_MASK)[(mb * 128 + j) * 2 + half];
+          keep[0] = kv.x;
+          keep[1] = kv.y;
+          mbar_arrive(bar_mask_empty(mb));
+        } else if constexpr (DROP) {
           // undropped P^T, and the keep bits from the dropped copy's zeros
           // (a kept entry whose P rounds to 0 has dS = 0 either way)
 #pragma unroll

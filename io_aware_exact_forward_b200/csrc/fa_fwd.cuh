@@ -23,8 +23,9 @@
 //   warp 8      MMA issuer (one thread): S_w = Q_w K_j^T into tensor memory,
 //               O_w += P_w V_j with P_w read from tensor memory.
 //   warps 10-11 no role (they complete the third warpgroup, whose registers
-//               go to the softmax warpgroups), except with dropout at d = 64,
-//               where they make each KV tile's keep bits for the softmax.
+//               go to the softmax warpgroups).
+//   warps 12-15 with dropout at d = 64 only: each KV tile's keep bits for the
+//               softmax, one warp per SM sub-partition.
 //   warps 0-3   softmax for query tile 0 (TMEM lanes 0..127, one row per
 //   warps 4-7   thread) and for query tile 1.  Each thread keeps m and l of
 //               its row in registers, writes P (bf16) over its S columns, and
@@ -55,9 +56,9 @@
 // Dropout variant (DROP = true, bf16): P is multiplied by a keep mask before
 // P V ("Efficient attention: memory-bound", "Real code moves even more", puts
 // dropout on the probabilities before the final product); the mask is
-// regenerated from Philox-4x32-10 for each tile (at d = 64 by warps 10-11,
-// which otherwise have no role, into shared memory; at d = 128 by the
-// softmax threads themselves), l sums the undropped P, and the epilogue
+// regenerated from Philox-4x32-10 for each tile (at d = 64 by a fourth
+// warpgroup, warps 12-15, into shared memory; at d = 128 by the softmax
+// threads themselves), l sums the undropped P, and the epilogue
 // scales O by 256 / t.
 //
 // The rescale is lazy: a row keeps its reference maximum until the running
@@ -104,8 +105,8 @@ struct FwdCfg {
   // E4M3: P0, P1 (128 rows x 128 one-byte keys each) in shared memory
   static constexpr int P_BYTES = BM * BN;
   static constexpr int OFF_P = OFF_RING + NSTAGE * TILE_BYTES;
-  // Dropout at d = 64: warps 10-11 (otherwise without a role) make each KV
-  // tile's keep bits ahead of the softmax, into two buffers of
+  // Dropout at d = 64: warps 12-15 make each KV tile's keep bits ahead of
+  // the softmax, into two buffers of
   // [2 query tiles][128 rows] x 128 bits; the softmax threads load their
   // row's 16 bytes.  (At d = 128 shared memory is full and the softmax
   // threads make their own.)
@@ -119,13 +120,18 @@ struct FwdCfg {
   static constexpr int NBAR = 4 + 2 * NSTAGE + 2 + 2 + 2 + 1 + 4 + (MASKW ? 4 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  static constexpr int THREADS = 384;
-  // setmaxnreg split of the launch's 384 x 168 registers: two softmax
-  // warpgroups at REG_SOFTMAX, the MMA/TMA warpgroup at REG_OTHER.
-  static constexpr int REG_LAUNCH = 168;
-  static constexpr int REG_SOFTMAX = 216;
-  static constexpr int REG_OTHER = 72;
-  static_assert(128 * (2 * REG_SOFTMAX + REG_OTHER) <= THREADS * REG_LAUNCH, "register split exceeds the launch");
+  // With the keep-bit warps a fourth warpgroup (warps 12-15) makes the bits,
+  // one warp on each SM sub-partition.
+  static constexpr int THREADS = MASKW ? 512 : 384;
+  static constexpr int MASK_THREADS = 128;
+  // setmaxnreg split of the launch's registers (384 x 168, or 512 x 128 with
+  // the keep-bit warpgroup): two softmax warpgroups at REG_SOFTMAX, the
+  // MMA/TMA warpgroup (and the keep-bit one) at REG_OTHER.
+  static constexpr int REG_LAUNCH = MASKW ? 128 : 168;
+  static constexpr int REG_SOFTMAX = MASKW ? 208 : 216;
+  static constexpr int REG_OTHER = MASKW ? 48 : 72;
+  static_assert(128 * (2 * REG_SOFTMAX + (THREADS / 128 - 2) * REG_OTHER) <= THREADS * REG_LAUNCH,
+                "register split exceeds the launch");
   static constexpr int TMEM_COLS = 512;
   // P apart from S, so that the next S can be computed as soon as the softmax
   // has loaded this one, overlapping the softmax: at d = 64 (bf16) in its own
@@ -187,7 +193,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
 }
 
 template <int D, bool F8 = false, bool DROP = false>
-__global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(FwdCfg<D, F8, DROP>::THREADS, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D, F8, DROP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
       mbar_init(bar_s_free(w), 128);
       mbar_init(bar_p_free(w), 1);
       if (C::MASKW) {
-        mbar_init(bar_mask_full(w), 64);
+        mbar_init(bar_mask_full(w), C::MASK_THREADS);
         mbar_init(bar_mask_empty(w), 256);
       }
     }
@@ -315,15 +321,16 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
         }
       }
     }
-  } else if (C::MASKW && warp >= 10) {
+  } else if (C::MASKW && warp >= 12) {
     // ------------------------------------------------------------ dropout mask
-    // Thread mt makes rows 4 (mt & 31) .. + 3 of query tile mt >> 5: for each
-    // of the tile's 32 key groups the Philox block of those four rows (the
-    // layout the softmax's own generator uses: counter (row / 4, key / 4, bh,
-    // offset), word = row, byte = key), each row's keep bits gathered into
-    // its four 32-key words.
-    const int mt = threadIdx.x - 320;
-    const int wq = mt >> 5, a_loc = mt & 31;
+    // Thread mt makes rows 4 a .. 4 a + 3 (a = (mt >> 1) & 31) of query tile
+    // mt >> 6 against key half mt & 1: for each of that half's 16 key groups
+    // the Philox block of those four rows (the layout the softmax's own
+    // generator uses: counter (row / 4, key / 4, bh, offset), word = row,
+    // byte = key), each row's keep bits gathered into its two 32-key words
+    // of the half.
+    const int mt = threadIdx.x - 384;
+    const int wq = mt >> 6, a_loc = (mt >> 1) & 31, kh = mt & 1;
     const uint32_t tt = p.drop_t * 0x01010101u;
     uint4* mbuf = reinterpret_cast<uint4*>(smem + C::OFF_MASK);
     bool ok = true;
@@ -340,7 +347,7 @@ __global__ void __launch_bounds__(384, 1) fa_fwd_kernel(const __grid_constant__ 
         const uint32_t c0 = (uint32_t)((it.kv0 + j) * C::BN) >> 2;
         uint32_t* mw = reinterpret_cast<uint32_t*>(mbuf + (buf * 2 + wq) * 128 + 4 * a_loc);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {  // keys 32k .. 32k + 31: eight Philox blocks
+        for (int k = 2 * kh; k < 2 * kh + 2; ++k) {  // keys 32k .. 32k + 31: eight Philox blocks
           uint32_t rw[4] = {0u, 0u, 0u, 0u};  // one word per row of the group
           // not unrolled: fully unrolled, the blocks' states spill at this
           // warpgroup's 72 registers (measured 1.37 against 1.19 ms)

@@ -470,14 +470,16 @@ static int dkdv_impl(const void* q, const void* k, const void* v, const void* dO
     return launch_status();
   }
   // deterministic: dK/dV without dQ, then the dQ pass
+  using C64 = BwdCfg<64, false, false>;
+  using C128 = BwdCfg<128, false, false>;
   if (d == 64 && window > 0)
-    fa_bwd_dkdv_kernel<64, true, false, false><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+    fa_bwd_dkdv_kernel<64, true, false, false><<<grid, C64::THREADS, C64::SMEM_BYTES, s>>>(p);
   else if (d == 64)
-    fa_bwd_dkdv_kernel<64, false, false, false><<<grid, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, s>>>(p);
+    fa_bwd_dkdv_kernel<64, false, false, false><<<grid, C64::THREADS, C64::SMEM_BYTES, s>>>(p);
   else if (window > 0)
-    fa_bwd_dkdv_kernel<128, true, false, false><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+    fa_bwd_dkdv_kernel<128, true, false, false><<<grid, C128::THREADS, C128::SMEM_BYTES, s>>>(p);
   else
-    fa_bwd_dkdv_kernel<128, false, false, false><<<grid, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, s>>>(p);
+    fa_bwd_dkdv_kernel<128, false, false, false><<<grid, C128::THREADS, C128::SMEM_BYTES, s>>>(p);
   if ((st = launch_status())) return st;
   if (Tq == 0) return FA_OK;
   DqParams qp;

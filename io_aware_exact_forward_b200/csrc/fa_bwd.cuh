@@ -164,7 +164,7 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 }
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-template <int D, bool DROP = false>
+template <int D, bool DROP = false, bool DQ = true>
 struct BwdCfg {
   static constexpr int NBOX = D / 64;
   static constexpr int BOX_BYTES = 128 * 128;
@@ -176,13 +176,14 @@ struct BwdCfg {
   // stages but a single dO buffer with its own barriers (the next dO is
   // loaded between this tile's dV and the next tile's dP^T), which leaves
   // room for two dQ staging boxes.  The staged boxes go out with bulk
-  // tensor reduce-adds.
+  // tensor reduce-adds.  Without dQ (DQ = false) the staging boxes' room
+  // holds a second dO buffer instead, and dO travels with Q in each stage.
   static constexpr int NSBUF = (D == 64) ? 2 : 1;
   static constexpr int NKV = (D == 64) ? 2 : 1;
-  static constexpr bool SPLIT_DO = (D == 128);
+  static constexpr bool SPLIT_DO = (D == 128) && DQ;
   static constexpr int NQ = (D == 64) ? 3 : 2;          // Q / LSE2 / D (and dO) stages
   static constexpr int NDO = SPLIT_DO ? 1 : NQ;         // dO buffers
-  static constexpr int NDQS = (D == 128) ? 2 : 1;       // dQ staging boxes
+  static constexpr int NDQS = (D == 128) ? 2 : 1;       // dQ staging boxes (none allocated without dQ)
   static constexpr int OFF_K = 0;                       // NKV buffers of (K, V)
   static constexpr int OFF_Q = 2 * NKV * TILE;          // NQ stages
   static constexpr int OFF_DO = OFF_Q + NQ * TILE;      // NDO buffers
@@ -190,7 +191,7 @@ struct BwdCfg {
   // fp32 staging of 32 dQ columns per box (128-byte swizzle), reused across
   // the boxes of the tile
   static constexpr int OFF_DQS = OFF_DS + 2 * BOX_BYTES;
-  static constexpr int DQS_BYTES = NDQS * 128 * 32 * 4;
+  static constexpr int DQS_BYTES = DQ ? NDQS * 128 * 32 * 4 : 0;
   static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;   // [NQ][128] f32
   static constexpr int OFF_DD = OFF_LSE + NQ * 128 * 4; // [NQ][128] f32
   // Dropout at d = 64: warps 22-23 make each query tile's keep bits ahead
@@ -305,7 +306,7 @@ __device__ __forceinline__ void dropout_keep_keyrow_64(uint32_t (&mask)[2], int 
 //   dV += (P*Z)^T dO * s,   dS = P * (Z * s * dP - D),   s = 256 / t.
 template <int D, bool WIN, bool DROP = false, bool DQ = true>
 __global__ void __maxnreg__(80) fa_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
-  using C = BwdCfg<D, DROP>;
+  using C = BwdCfg<D, DROP, DQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {  // the layout needs 1024-byte aligned swizzle atoms
@@ -983,10 +984,16 @@ static int bwd_setup() {
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<64, true, false, false>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, false, false, false>),
                             reinterpret_cast<const void*>(fa_bwd_dkdv_kernel<128, true, false, false>)};
-  const int bytes[10] = {BwdCfg<64>::SMEM_BYTES,       BwdCfg<64>::SMEM_BYTES,       BwdCfg<128>::SMEM_BYTES,
-                         BwdCfg<128>::SMEM_BYTES,      BwdCfg<64, true>::SMEM_BYTES, BwdCfg<128, true>::SMEM_BYTES,
-                         BwdCfg<64>::SMEM_BYTES,       BwdCfg<64>::SMEM_BYTES,       BwdCfg<128>::SMEM_BYTES,
-                         BwdCfg<128>::SMEM_BYTES};
+  const int bytes[10] = {BwdCfg<64>::SMEM_BYTES,
+                         BwdCfg<64>::SMEM_BYTES,
+                         BwdCfg<128>::SMEM_BYTES,
+                         BwdCfg<128>::SMEM_BYTES,
+                         BwdCfg<64, true>::SMEM_BYTES,
+                         BwdCfg<128, true>::SMEM_BYTES,
+                         BwdCfg<64, false, false>::SMEM_BYTES,
+                         BwdCfg<64, false, false>::SMEM_BYTES,
+                         BwdCfg<128, false, false>::SMEM_BYTES,
+                         BwdCfg<128, false, false>::SMEM_BYTES};
   for (int i = 0; i < 10; ++i)
     if (cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes[i]) != cudaSuccess)
       return FA_ERR_CUDA;

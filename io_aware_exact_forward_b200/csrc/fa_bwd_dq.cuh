@@ -19,7 +19,7 @@
 // Warp roles (320 threads): 0-7 compute (two warps per TMEM lane quarter,
 // one per half of the 128 key columns; one query row per lane), 8 MMA issuer,
 // 9 TMA producer.  Tensor memory: S [0,128), dP [128,256), dQ [256,256+d),
-// dS (bf16 pairs) [256+d, 320+d).  Shared memory: Q and dO (one tile each)
+// two dS buffers (bf16 pairs) [256+d, 384+d).  Shared memory: Q and dO (one tile each)
 // and a ring of two (K_j, V_j) stages.  S_{j+1} and dP_{j+1} are issued as
 // soon as the compute warps have loaded S_j and dP_j, so the products of the
 // next tile overlap the exponentials of this one.
@@ -56,9 +56,9 @@ struct DqCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_DO = TILE;
   static constexpr int OFF_RING = 2 * TILE;
-  // qdo_full, kv_full[NST], kv_empty[NST], s_full, s_free, ds_full, ds_free,
-  // dq_done, mma_done
-  static constexpr int NBAR = 1 + 2 * NST + 6;
+  // qdo_full, kv_full[NST], kv_empty[NST], s_full, s_free, ds_full[2],
+  // ds_free[2], dq_done, mma_done
+  static constexpr int NBAR = 1 + 2 * NST + 8;
   static constexpr int OFF_BAR = OFF_RING + NST * 2 * TILE;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // tmem base (u32), abort flag (int)
   // + alignment slack; at least 120 KB, so that two CTAs never share an SM
@@ -69,10 +69,10 @@ struct DqCfg {
   static constexpr int TM_S = 0;
   static constexpr int TM_DP = 128;
   static constexpr int TM_DQ = 256;
-  static constexpr int TM_DS = 256 + D;
+  static constexpr int TM_DS = 256 + D;            // two dS buffers of 64 columns
   static constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 0, 1);   // dS from TMEM, K MN-major
-  static_assert(TM_DS + 64 <= TMEM_COLS, "tensor memory overflow");
+  static_assert(TM_DS + 128 <= TMEM_COLS, "tensor memory overflow");
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
 };
 
@@ -122,10 +122,12 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dq_kernel(const __grid_constant
   auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + C::NST + s); };
   const uint32_t bar_s_full = bar0 + 8u * (1 + 2 * C::NST);   // S_j and dP_j in tensor memory
   const uint32_t bar_s_free = bar0 + 8u * (2 + 2 * C::NST);   // the compute warps hold them
-  const uint32_t bar_ds_full = bar0 + 8u * (3 + 2 * C::NST);  // dS_j in tensor memory
-  const uint32_t bar_ds_free = bar0 + 8u * (4 + 2 * C::NST);  // dQ += dS_j K_j has read it
-  const uint32_t bar_dq_done = bar0 + 8u * (5 + 2 * C::NST);
-  const uint32_t bar_mma_done = bar0 + 8u * (6 + 2 * C::NST);
+  // dS of tile j in buffer j & 1; a barrier pair per buffer, so that no
+  // wait is ever for a phase two behind
+  auto bar_ds_full = [&](int b) { return bar0 + 8u * (3 + 2 * C::NST + b); };  // dS_j in tensor memory
+  auto bar_ds_free = [&](int b) { return bar0 + 8u * (5 + 2 * C::NST + b); };  // dQ += dS_j K_j has read it
+  const uint32_t bar_dq_done = bar0 + 8u * (7 + 2 * C::NST);
+  const uint32_t bar_mma_done = bar0 + 8u * (8 + 2 * C::NST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   const uint32_t aQ = sbase + C::OFF_Q, aDO = sbase + C::OFF_DO;
@@ -146,8 +148,10 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dq_kernel(const __grid_constant
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_s_free, 256);
-    mbar_init(bar_ds_full, 256);
-    mbar_init(bar_ds_free, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_ds_full(b), 256);
+      mbar_init(bar_ds_free(b), 1);
+    }
     mbar_init(bar_dq_done, 1);
     mbar_init(bar_mma_done, 1);
     fence_barrier_init();
@@ -225,12 +229,13 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dq_kernel(const __grid_constant
           if (j > 0) {
             // dQ += dS_{j-1} K_{j-1}, then the stage and the dS columns are free
             const int s = (j - 1) % C::NST;
-            ok = mbar_wait(bar_ds_full, (j - 1) & 1, wc);
+            ok = mbar_wait(bar_ds_full((j - 1) & 1), ((j - 1) >> 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mma_ts(tDQ, tDS + 8 * k, mndesc(aK(s), k), C::IDESC_DQ, j > 1 || k > 0);
-            mma_commit(bar_ds_free);
+            for (int k = 0; k < 8; ++k)
+              mma_ts(tDQ, tDS + 64 * ((j - 1) & 1) + 8 * k, mndesc(aK(s), k), C::IDESC_DQ, j > 1 || k > 0);
+            mma_commit(bar_ds_free((j - 1) & 1));
             mma_commit(bar_kv_empty(s));
           }
         }
@@ -289,16 +294,16 @@ __global__ void __launch_bounds__(320, 1) fa_bwd_dq_kernel(const __grid_constant
         const float2 g = __fmul2_rn(pr, t);
         ds[e] = pack_bf16x2(g.x, g.y);
       }
-      // the dS columns are free once the previous tile's dQ product has read them
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_ds_free, (j - 1) & 1, wc));
+      // dS buffer j & 1 is free once the dQ product of tile j - 2 has read it
+      if (j > 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_ds_free(j & 1), ((j - 2) >> 1) & 1, wc));
         if (!ok) break;
       }
       tc_fence_after();
-      tmem_st32(tDS, ds);
+      tmem_st32(tDS + 64 * (j & 1), ds);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_ds_full);
+      mbar_arrive(bar_ds_full(j & 1));
     }
     // ------------------------------------------------------------ epilogue
     if (ok && it.n_kv > 0) {

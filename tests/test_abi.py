@@ -223,3 +223,18 @@ def test_every_exported_symbol_is_declared():
     out = subprocess.run([nm, "-D", "--defined-only", fa.LIB_PATH], capture_output=True, text=True, check=True).stdout
     exported = sorted({ln.split()[-1] for ln in out.splitlines() if ln.split() and ln.split()[-1].startswith("fa_")})
     assert exported == _header_functions()
+
+
+def test_deterministic_backward_argument_checks():
+    lib = fa.load_library()
+    args = [NULL] * 9 + [NULL, 0]
+    # a window needs causal = 1, and must not be negative
+    assert lib.fa_backward_deterministic(*args, 1, 1, 1, 16, 16, 64, 1.0, 0, 8, NULL) == 1
+    assert lib.fa_backward_deterministic(*args, 1, 1, 1, 16, 16, 64, 1.0, 1, -1, NULL) == 1
+    # the shared prefill checks: GQA divisibility, head size, finite scale
+    assert lib.fa_backward_deterministic(*args, 1, 3, 2, 16, 16, 64, 1.0, 1, 0, NULL) == 1
+    assert lib.fa_backward_deterministic(*args, 1, 1, 1, 16, 16, 96, 1.0, 1, 0, NULL) == 2
+    assert lib.fa_backward_deterministic(*args, 1, 1, 1, 16, 16, 64, float("nan"), 0, 0, NULL) == 1
+    # null pointers are rejected; an empty problem is a no-op
+    assert lib.fa_backward_deterministic(*args, 1, 1, 1, 16, 16, 64, 1.0, 1, 0, NULL) == 1
+    assert lib.fa_backward_deterministic(*args, 0, 1, 1, 16, 16, 64, 1.0, 1, 0, NULL) == 0

@@ -58,3 +58,73 @@ def test_random_shape(i, B, Hq, Hkv, Tq, Tk, d, causal, window):
         assert_grad_close(to_f64(y), r, name + " (deterministic)")
     # dK and dV are the same bits either way
     assert torch.equal(grads[1], det[1]) and torch.equal(grads[2], det[2])
+
+
+def _draw_dropout(n, seed=977):
+    rng = random.Random(seed)
+    cases = []
+    for i in range(n):
+        hkv = rng.choice([1, 2])
+        g = rng.choice([1, 2, 4])
+        tq = rng.randint(1, 600)
+        tk = tq if rng.random() < 0.5 else rng.randint(1, 600)
+        cases.append((i, rng.choice([1, 2]), hkv * g, hkv, tq, tk, rng.choice([64, 128]), rng.random() < 0.5,
+                      rng.choice([0.05, 0.1, 0.3, 0.6])))
+    return cases
+
+
+@pytest.mark.parametrize("i,B,Hq,Hkv,Tq,Tk,d,causal,p", _draw_dropout(12))
+def test_random_shape_dropout(i, B, Hq, Hkv, Tq, Tk, d, causal, p):
+    """fa_forward_dropout and fa_backward_dropout against the oracle's
+    attention with the same Philox mask (O compared after undoing the
+    256/t scale both sides apply)."""
+    from oracle import dropout as dr
+    w = WORKLOADS[1].with_(B=B, Hq=Hq, Hkv=Hkv, d=d, causal=causal)
+    inp = prefill_inputs(w, seed=3000 + i, Tq=Tq, Tk=Tk)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "do"))
+    seed, offset = 0x51DE_0000 + 17 * i, 5 + i
+    o, lse = fa.forward_dropout(q, k, v, p, seed, offset, scale=w.scale, causal=causal)
+    dq, dk, dv = fa.backward_dropout(q, k, v, o, lse, do, p, seed, offset, scale=w.scale, causal=causal)
+    torch.cuda.synchronize()
+    assert fa.check() == 0
+    f64 = {n: to_f64(inp[n]) for n in ("q", "k", "v", "do")}
+    O, LSE = dr.attention_forward_dropout(f64["q"], f64["k"], f64["v"], w.scale, causal, p, seed, offset)
+    back = dr.keep_threshold(p) / 256.0
+    assert_o_close(to_f64(o) * back, O * back)
+    assert_lse_close(lse.cpu().numpy(), LSE)
+    R = dr.attention_backward_dropout(f64["q"], f64["k"], f64["v"], f64["do"], w.scale, causal, p, seed, offset)
+    for name, x, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), R):
+        assert_grad_close(to_f64(x), r, name)
+
+
+def _draw_decode(n, seed=4242):
+    rng = random.Random(seed)
+    cases = []
+    for i in range(n):
+        hkv = rng.choice([1, 2, 4])
+        g = rng.choice([1, 2, 4, 8])
+        tk_max = rng.randint(1, 1500)
+        b = rng.randint(1, 5)
+        seqlens = [rng.choice([0, rng.randint(1, tk_max), tk_max]) for _ in range(b)]
+        window = rng.choice([None, None, 1, 100, 700])
+        cases.append((i, hkv * g, hkv, rng.choice([64, 128]), rng.choice([64, 128, 256, 512]), tk_max, seqlens,
+                      window))
+    return cases
+
+
+@pytest.mark.parametrize("i,Hq,Hkv,d,chunk,Tk_max,seqlens,window", _draw_decode(12))
+def test_random_shape_decode(i, Hq, Hkv, d, chunk, Tk_max, seqlens, window):
+    """Split-KV decode (optionally windowed) against the oracle's one-token
+    forward over each sequence's first seqlens[b] keys."""
+    from workloads import decode_inputs
+    w = WORKLOADS[5].with_(Hq=Hq, Hkv=Hkv, d=d)
+    inp = decode_inputs(w, seed=5000 + i, B=len(seqlens), Tk_max=Tk_max, seqlens=seqlens)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o, lse = fa.decode_splitkv(dev["q"], dev["k_cache"], dev["v_cache"], dev["seqlens"], scale=w.scale,
+                               chunk=chunk, window=window)
+    torch.cuda.synchronize()
+    assert fa.check() == 0
+    O, LSE = oracle.decode_forward(to_f64(inp["q"]), to_f64(inp["k_cache"]), to_f64(inp["v_cache"]),
+                                   inp["seqlens"].cpu().numpy(), w.scale, window=window)
+    assert_o_close(to_f64(o), O)
+    assert_lse_close(lse.cpu().numpy(), LSE)

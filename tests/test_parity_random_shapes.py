@@ -128,3 +128,33 @@ def test_random_shape_decode(i, Hq, Hkv, d, chunk, Tk_max, seqlens, window):
                                    inp["seqlens"].cpu().numpy(), w.scale, window=window)
     assert_o_close(to_f64(o), O)
     assert_lse_close(lse.cpu().numpy(), LSE)
+
+
+def _draw_fp8(n, seed=808):
+    rng = random.Random(seed)
+    cases = []
+    for i in range(n):
+        hkv = rng.choice([1, 2])
+        g = rng.choice([1, 2, 4])
+        tq = rng.randint(1, 700)
+        tk = tq if rng.random() < 0.5 else rng.randint(1, 700)
+        cases.append((i, rng.choice([1, 2]), hkv * g, hkv, tq, tk, rng.random() < 0.6))
+    return cases
+
+
+@pytest.mark.parametrize("i,B,Hq,Hkv,Tq,Tk,causal", _draw_fp8(8))
+def test_random_shape_fp8(i, B, Hq, Hkv, Tq, Tk, causal):
+    """fa_forward_fp8 (d = 128) against the oracle on the dequantised inputs,
+    each element under the bound E4M3 rounding of P allows."""
+    from workloads import prefill_inputs_e4m3
+    from test_parity_fp8 import _check_head
+    w = WORKLOADS[3].with_(B=B, Hq=Hq, Hkv=Hkv, causal=causal)
+    inp = prefill_inputs_e4m3(w, seed=7000 + i, Tq=Tq, Tk=Tk)
+    dev = {n: (t.cuda() if torch.is_tensor(t) else t) for n, t in inp.items()}
+    o, lse = fa.forward_fp8(dev["q"], dev["k"], dev["v"], inp["q_descale"], inp["k_descale"], inp["v_descale"],
+                            scale=w.scale, causal=causal)
+    torch.cuda.synchronize()
+    assert fa.check() == 0
+    for b in range(B):
+        for h in range(Hq):
+            _check_head(o, lse, inp, b, h, Hq // Hkv, w.scale, causal)

@@ -41,6 +41,8 @@
 // (two warps per TMEM lane quarter, one per half of the 128 query columns);
 // 16-19 dQ read-out and reduce-adds (one query row per thread); 20 MMA
 // issuer; 21 TMA producer; with dropout at d = 64, 22-23 make the keep bits.
+// The deterministic backward builds dkdv without dQ (DQ = false: no dQ
+// product, warps 16-19 idle) and takes dQ from the pass in fa_bwd_dq.cuh.
 #pragma once
 
 #include "fa_ptx.cuh"

@@ -63,6 +63,9 @@ def parse_args():
                          "fa_backward_dkdv_dropout)")
     ap.add_argument("--cp", action="store_true",
                     help="decode only: context-parallel, every sequence's cache cut into one share per GPU")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="prefill: forward + fa_backward_deterministic (dQ from its own pass, the same bits on "
+                         "every run); the default step is timed beside it")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (smaller cases for profiler captures only)")
     return ap.parse_args()
@@ -1144,6 +1147,97 @@ def run_dropout(args, w, rank, world, dist):
     return 0
 
 
+def run_deterministic(args, w, rank, world, dist):
+    """Forward + the deterministic backward (fa_backward_deterministic: the
+    preprocess, the dK/dV kernel without dQ and the dQ pass in one call) on a
+    prefill workload, inputs resident and larger than L2; the default step
+    (fused dQ) is timed the same way in the same run for comparison."""
+    import torch
+    import io_aware_exact_forward_b200 as fa
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = fa.load_library()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    run = _PrefillRun(lib, fa, w, dev, w.seed + rank)
+    B, Hq, Hkv, T, d = w.B, w.Hq, w.Hkv, w.T, w.d
+    causal, window = int(w.causal or bool(w.window)), int(w.window or 0)
+
+    def step(evs=None):
+        s = run.stream
+        if evs: evs[0].record(s)
+        run._check(run.fwd_fn(run.pq, run.pk, run.pv, run.po, run.plse, B, Hq, Hkv, T, T, d, w.scale,
+                              run.mask_arg, run.sp), "fa_forward")
+        if evs: evs[1].record(s)
+        run._check(lib.fa_backward_deterministic(run.pq, run.pk, run.pv, run.po, run.plse, run.pdo, run.pdq, run.pdk,
+                                                 run.pdv, run.pws, run.ws_bytes, B, Hq, Hkv, T, T, d, w.scale,
+                                                 causal, window, run.sp), "fa_backward_deterministic")
+        if evs: evs[2].record(s)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if lib.fa_check(run.sp) != 0:
+        raise RuntimeError("device status set during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(run.stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(run.stream)
+        barrier()
+    if lib.fa_check(run.sp) != 0:
+        raise RuntimeError("device status set in the timed region")
+    elapsed = t0.elapsed_time(t1)
+    seg = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(2)]
+    elapsed_plain, seg_plain = run.timed(args.steps, args.warmup, barrier)
+    del run
+    elapsed = max_over_ranks(elapsed, dist, dev)
+    elapsed_plain = max_over_ranks(elapsed_plain, dist, dev)
+    f_fwd, f_bwd = flops(w)
+    value = job_rate(f_fwd + f_bwd, world, args.steps, elapsed) / 1e12
+    ms = elapsed / args.steps
+    peaks = load_peaks()
+    bwd_name = "fa_backward_deterministic (preprocess, dK/dV without dQ, dQ pass)"
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "tokens_per_s": world * prefill_tokens(w) / (ms * 1e-3),
+            "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d, "causal": w.causal,
+                       "window": w.window or None,
+                       "step": "fa_forward + fa_backward_deterministic", "l2": "inputs larger than L2",
+                       "seed": w.seed},
+            "per_kernel_ms": {"fa_fwd_kernel": seg[0], bwd_name: seg[1]},
+            "default": {"ms_per_step": elapsed_plain / args.steps,
+                        "tflops": job_rate(f_fwd + f_bwd, world, args.steps, elapsed_plain) / 1e12,
+                        "per_kernel_ms": seg_plain},
+            # the backward is one call of three launches: its roofline is the
+            # call's, against the tensor peak
+            "roofline": {"kernel": bwd_name, "bound": "tensor", "achieved": f_bwd / (seg[1] * 1e-3) / 1e12,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": f_bwd / (seg[1] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                         "peak_source": f"{peaks['source']} bf16 dense (burst)", "traffic": None,
+                         "algorithmic_per_launch": f_bwd},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks.summary(),
+            "cpu_baseline": None,
+            "e2e": None,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_decode_cp(args, w, rank, world, dist):
     """Context-parallel decode of the same batch: every sequence's cache is
     cut into `world` contiguous shares and rank r holds share r.  One step is
@@ -1292,6 +1386,9 @@ def main():
         print("--dropout takes a rate in [0, 1) and applies to the prefill workloads without a window",
               file=sys.stderr)
         return 2
+    if args.deterministic and (w.decode or args.fp8 or args.dropout is not None):
+        print("--deterministic applies to the plain prefill workloads (no --fp8 or --dropout)", file=sys.stderr)
+        return 2
     if args.cp and (not w.decode or w.window):
         print("--cp applies to the decode workload without a window", file=sys.stderr)
         return 2
@@ -1312,6 +1409,8 @@ def main():
             return run_fp8_forward(args, w, rank, world, dist)
         if args.dropout is not None:
             return run_dropout(args, w, rank, world, dist)
+        if args.deterministic:
+            return run_deterministic(args, w, rank, world, dist)
         if w.decode and args.cp:
             return run_decode_cp(args, w, rank, world, dist)
         if w.decode:

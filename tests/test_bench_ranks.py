@@ -57,3 +57,15 @@ def test_pair_count_matches_brute_force():
         for W in (1, 2, 7, 128, 1000):
             brute = sum(1 for i in range(Tq) for j in range(Tk) if i + Tk - Tq - W < j <= i + Tk - Tq)
             assert bench.pairs_count(Tq, Tk, True, W) == brute
+
+
+def test_incompatible_modes_are_refused_before_any_device_work(monkeypatch, capsys):
+    """Mode combinations bench.py does not run return status 2 from the
+    argument checks, which come before anything touches a GPU."""
+    import sys
+    import bench
+    for argv in (["--deterministic", "--fp8", "--workload", "3"], ["--deterministic", "--dropout", "0.1"],
+                 ["--deterministic", "--workload", "5"], ["--fp8"], ["--dropout", "1.5"], ["--cp"],
+                 ["--window", "0"]):
+        monkeypatch.setattr(sys, "argv", ["bench.py"] + argv)
+        assert bench.main() == 2, argv
